@@ -1,0 +1,196 @@
+"""The oracle's attention against things other than itself.
+
+Pins:
+* a library routine: torch's scaled_dot_product_attention in float64 on the
+  CPU, with grouped-query heads expanded by repeat_interleave (query head h
+  reads KV head h // G), on contiguous histories;
+* closed-form special cases: length 1 gives v_0, equal keys give the mean of
+  V, one dominant logit gives that token's v, length 0 gives 0;
+* invariances the pages ask for: randomly permuted physical block ids, slots
+  past the length poisoned with NaN;
+* the paged online recurrence and the merge of split states against the dense
+  definition in binary64 (P3's executed check reports 2.22e-16 over 8 cases);
+* extreme logits (|s| ~ 1e3) stay finite and agree.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as att
+from oracle import kvops
+from oracle.allocator import OK, RefAllocator
+from tests.conftest import golden
+from workloads import normal_bf16_bits, normal_f32, rng
+
+
+def _sdpa_f64(q, K, V, scale):
+    """q [H_q, d], K/V [n, H_kv, d] float64 -> [H_q, d] via torch SDPA."""
+    H_q = q.shape[0]
+    H_kv = K.shape[1]
+    G = H_q // H_kv
+    qt = torch.from_numpy(q)[:, None, :]                     # [H_q, 1, d]
+    kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(G, dim=0)  # [H_q, n, d]
+    vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(G, dim=0)
+    out = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None], scale=scale)
+    return out[0, :, 0, :].numpy()
+
+
+@pytest.mark.parametrize("n,H_q,H_kv,d", [(1, 4, 1, 8), (5, 8, 2, 16), (37, 8, 2, 64), (200, 32, 8, 128),
+                                          (17, 16, 4, 32), (64, 32, 4, 128)])
+def test_dense_matches_torch_sdpa(n, H_q, H_kv, d):
+    g = rng(100 + n)
+    q = normal_f32(g, (H_q, d)).astype(np.float64)
+    K = normal_f32(g, (n, H_kv, d)).astype(np.float64)
+    V = normal_f32(g, (n, H_kv, d)).astype(np.float64)
+    scale = 1.0 / np.sqrt(d)
+    ref = _sdpa_f64(q, K, V, scale)
+    out = att.dense_decode(q, K, V, scale)
+    assert np.max(np.abs(out - ref)) < 1e-13
+
+
+def test_length_one_returns_v0():
+    g = rng(1)
+    q = normal_bf16_bits(g, (8, 64))
+    K = normal_bf16_bits(g, (1, 2, 64))
+    V = normal_bf16_bits(g, (1, 2, 64))
+    out = att.dense_decode(q, K, V, 0.125)
+    Vf = att.widen(V)
+    for h in range(8):
+        assert np.array_equal(out[h], Vf[0, h // 4])
+
+
+def test_length_zero_is_zero():
+    out = att.dense_decode(np.ones((4, 8), np.float32), np.zeros((0, 2, 8), np.float32),
+                           np.zeros((0, 2, 8), np.float32), 0.5)
+    assert np.array_equal(out, np.zeros((4, 8)))
+
+
+def test_equal_keys_give_mean_of_values():
+    g = rng(2)
+    n, H_kv, d = 50, 2, 16
+    q = normal_f32(g, (4, d))
+    K = np.repeat(normal_f32(g, (1, H_kv, d)), n, axis=0)
+    V = normal_f32(g, (n, H_kv, d))
+    out = att.dense_decode(q, K, V, 0.25)
+    for h in range(4):
+        np.testing.assert_allclose(out[h], V.astype(np.float64)[:, h // 2].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_dominant_logit_selects_value():
+    g = rng(3)
+    n, d = 40, 32
+    K = normal_f32(g, (n, 1, d))
+    V = normal_f32(g, (n, 1, d))
+    star = 17
+    q = (K[star, 0] * 1000.0)[None, :]
+    out = att.dense_decode(q, K, V, 1.0)
+    np.testing.assert_allclose(out[0], V[star, 0].astype(np.float64), rtol=0, atol=1e-12)
+
+
+def _paged_setup(lengths, B, H_kv, d, seed, dtype="f32", poison=True):
+    g = rng(seed)
+    nb = sum(-(-n // B) for n in lengths) + 3
+    perm = g.permutation(nb)
+    a = RefAllocator(nb, B, free_order=perm)
+    for i, n in enumerate(lengths):
+        assert a.add_seq(i, n) == OK
+    if dtype == "f32":
+        fill = np.nan if poison else 0.0
+        kp = kvops.new_pool(nb, B, H_kv, d, np.float32, fill)
+        vp = kvops.new_pool(nb, B, H_kv, d, np.float32, fill)
+        hk = [normal_f32(g, (n, H_kv, d)) for n in lengths]
+        hv = [normal_f32(g, (n, H_kv, d)) for n in lengths]
+    else:
+        fill = 0x7FC0 if poison else 0
+        kp = kvops.new_pool(nb, B, H_kv, d, np.uint16, fill)
+        vp = kvops.new_pool(nb, B, H_kv, d, np.uint16, fill)
+        hk = [normal_bf16_bits(g, (n, H_kv, d)) for n in lengths]
+        hv = [normal_bf16_bits(g, (n, H_kv, d)) for n in lengths]
+    for i in range(len(lengths)):
+        kvops.scatter_history(kp, a.table(i), hk[i])
+        kvops.scatter_history(vp, a.table(i), hv[i])
+    tables = [a.table(i) for i in range(len(lengths))]
+    return kp, vp, tables, hk, hv
+
+
+@pytest.mark.parametrize("B", [4, 16, 64])
+def test_permuted_blocks_and_poisoned_tails_match_dense(B):
+    """Random physical ids, NaN in every unwritten slot, lengths 0/1/B/B+1 and more."""
+    lengths = [0, 1, B, B + 1, 37, 91, 2 * B - 1]
+    H_q, H_kv, d = 8, 2, 16
+    kp, vp, tables, hk, hv = _paged_setup(lengths, B, H_kv, d, seed=B)
+    g = rng(500 + B)
+    q = normal_f32(g, (len(lengths), H_q, d))
+    scale = 1 / 4
+    out = att.paged_decode(q, kp, vp, tables, lengths, scale)
+    assert np.all(np.isfinite(out))
+    for i, n in enumerate(lengths):
+        ref = _sdpa_f64(q[i].astype(np.float64), hk[i].astype(np.float64), hv[i].astype(np.float64), scale) \
+            if n > 0 else np.zeros((H_q, d))
+        assert np.max(np.abs(out[i] - ref)) < 1e-13
+        online = att.paged_online_decode(q[i], kp, vp, tables[i], n, scale)
+        assert np.all(np.isfinite(online))
+        assert np.max(np.abs(online - out[i])) < 1e-14
+
+
+def test_online_recurrence_matches_dense_witness():
+    """P3's executed check: binary64 online softmax vs dense over 8 cases and several block sizes."""
+    w = golden("witness.json")
+    worst = 0.0
+    cases = 0
+    for case in range(w["attention_cases"]):
+        g = rng(900 + case)
+        n = int(g.integers(1, 300))
+        q = normal_f32(g, (4, 32)).astype(np.float64)
+        K = normal_f32(g, (n, 2, 32)).astype(np.float64)
+        V = normal_f32(g, (n, 2, 32)).astype(np.float64)
+        dense = att.dense_decode(q, K, V, 1 / np.sqrt(32))
+        for blk in (1, 4, 16, 64):
+            online = att.online_decode_blocks(q, K, V, 1 / np.sqrt(32), blk)
+            worst = max(worst, float(np.max(np.abs(online - dense))))
+        cases += 1
+    assert cases == w["attention_cases"]
+    # same order of magnitude as the printed 2.22e-16: a few ulps of |out| <= 1
+    assert worst <= 8 * w["largest_absolute_error"]
+
+
+def test_merge_of_split_states_matches_dense():
+    g = rng(11)
+    n = 777
+    q = normal_f32(g, (8, 64))
+    K = normal_f32(g, (n, 2, 64))
+    V = normal_f32(g, (n, 2, 64))
+    dense = att.dense_decode(q, K, V, 0.125)
+    for cuts in ([0, n], [0, 1, n], [0, 100, 100, 400, n], list(range(0, n, 64)) + [n]):
+        merged = att.finish(att.merge_states(att.split_states(q, K, V, 0.125, cuts)))
+        assert np.max(np.abs(merged - dense)) < 1e-14
+
+
+def test_equal_weight_average_of_blocks_is_wrong():
+    """P2's third exercise: averaging per-block softmax outputs loses the normalisation."""
+    g = rng(12)
+    n = 40
+    q = normal_f32(g, (1, 16), 3.0)
+    K = normal_f32(g, (n, 1, 16))
+    V = normal_f32(g, (n, 1, 16))
+    dense = att.dense_decode(q, K, V, 0.25)
+    per_block = [att.dense_decode(q, K[a:a + 16], V[a:a + 16], 0.25) for a in range(0, n, 16)]
+    assert np.max(np.abs(np.mean(per_block, axis=0) - dense)) > 1e-3
+
+
+@pytest.mark.parametrize("qscale", [30.0, 1000.0])
+def test_extreme_logits_stay_finite(qscale):
+    g = rng(13)
+    n, d = 300, 128
+    q = normal_bf16_bits(g, (32, d), qscale)
+    K = normal_bf16_bits(g, (n, 8, d))
+    V = normal_bf16_bits(g, (n, 8, d))
+    scale = 1 / np.sqrt(d)
+    dense = att.dense_decode(q, K, V, scale)
+    assert np.all(np.isfinite(dense))
+    s = scale * np.einsum("hd,nhd->hn", att.widen(q), np.repeat(att.widen(K), 4, axis=1))
+    assert np.max(np.abs(s)) > qscale      # logits of order qscale (|s| ~ 1e3 at x1000)
+    ref = _sdpa_f64(att.widen(q), att.widen(K), att.widen(V), scale)
+    assert np.max(np.abs(dense - ref)) < 1e-12
+    online = att.online_decode_blocks(q, K, V, scale, 16)
+    assert np.max(np.abs(online - dense)) < 1e-12
