@@ -1,0 +1,501 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark of the paged KV-cache hot path on B200.
+
+One step = one decode iteration of the teaching-model workload: 32 layers,
+32 requests with a 4096-token history (growing by one token per step),
+H_q 32 / H_kv 8 / d 128, bf16 K/V/Q, block size 16, block tables over a
+shuffled pool of 16 GiB + 10 %.  Per step:
+  host allocator append (C++; allocate-or-fail) -> block tables mirrored to
+  the device (pinned double buffer) -> copy-on-write copies if any -> slot
+  mapping -> decode plan -> for each layer: kv_append + paged decode attention.
+
+Reported (one JSON line from rank 0):
+  value        algorithmic HBM bytes of the step / device step time (GB/s);
+               bytes = K/V history read once per KV head + q + out + new
+               K/V written + block tables and lengths
+  e2e          the same metric with q, new K/V from pinned host buffers and
+               the outputs read back to the host inside the timed region
+  roofline     paged decode attention (partition + merge kernels) bytes per
+               launch / its CUDA-event duration, against the measured HBM peak
+  cpu_baseline the float64 oracle on the host cores, on a bounded sample
+  clocks       nvidia-smi samples taken during the timed region
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 it runs under torchrun, one rank per GPU, each rank serving its own
+32 x 4096 batch (weak scaling; no collective on the data path, only the
+barrier and the max-over-ranks of the step time).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "paged decode-attn achieved HBM GB/s (frac of peak); decode steps/s at 32x4096"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--seed", type=int, default=1)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# -- distributed plumbing -------------------------------------------------------
+def dist_init(n):
+    if n <= 1:
+        return 0, 1, None
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ["RANK"])
+    world = int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, dist
+
+
+def _reduce(x: float, dist, op: str, device: str) -> float:
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def max_over_ranks(x: float, dist, device: str = "cuda") -> float:
+    """The slowest rank's time: a multi-GPU number is timed as the max over ranks."""
+    return _reduce(x, dist, "max", device)
+
+
+def sum_over_ranks(x: float, dist, device: str = "cuda") -> float:
+    return _reduce(x, dist, "sum", device)
+
+
+def shard_requests(num_requests: int, world: int, rank: int) -> range:
+    """Requests served by one rank: each rank owns a disjoint, equal block of
+    request ids (weak scaling: per-rank work is fixed, the total grows with N).
+    Requests are independent, so ranks exchange nothing on the data path."""
+    return range(rank * num_requests, (rank + 1) * num_requests)
+
+
+# -- clocks -----------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str):
+        self.uuid = device_uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "samples": len(sm),
+                "power_w_max": float(max(power)) if power else None, "reasons": sorted(reasons)}
+
+
+# -- the workload -------------------------------------------------------------------
+class DecodeStep:
+    """32-layer decode step through the C ABI; all state resident on the device."""
+
+    def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1):
+        import torch
+
+        import paged_kv_cache_358_b200 as pkv
+        import workloads as W
+
+        self.torch, self.pkv = torch, pkv
+        pkv.set_decode_kernel(kernel)
+        wl = W.workload("teaching_32x4096", decode_steps=steps_budget + 8, seed=seed)
+        self.wl = wl
+        S, L, Hq, Hkv, D, B = wl.num_seqs, wl.layers, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+        self.S, self.L, self.Hq, self.Hkv, self.D, self.B = S, L, Hq, Hkv, D, B
+        N = wl.pool_blocks
+        self.N = N
+        g = W.rng(seed)
+        order = W.free_order(g, N)
+        self.alloc = pkv.BlockAllocator(N, B, free_order=order)
+        self.ids = np.array(list(shard_requests(S, world, rank)), dtype=np.int32)
+        for i, n in zip(self.ids, wl.lengths):
+            assert self.alloc.add_seq(int(i), n) == 0
+        self.max_blocks = -(-(max(wl.lengths) + steps_budget + 8) // B)
+        dev = torch.device("cuda")
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        shape = (N, B, Hkv, D)
+        self.k_pools, self.v_pools = [], []
+        for _ in range(L):
+            self.k_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+            self.v_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+        self.q = [torch.randn((S, Hq, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        self.k_new = [torch.randn((S, Hkv, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        self.v_new = [torch.randn((S, Hkv, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        self.out = [torch.empty((S, Hq, D), device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        self.status = np.zeros(S, dtype=np.int32)
+        self.copies_h = np.zeros((S, 3), dtype=np.int32)
+        # pinned double buffers for the tables and lengths mirrored each step
+        self.tab_h = [torch.empty((S, self.max_blocks), dtype=torch.int32).pin_memory() for _ in range(2)]
+        self.len_h = [torch.empty((S,), dtype=torch.int32).pin_memory() for _ in range(2)]
+        self.pos_h = [torch.empty((S,), dtype=torch.int32).pin_memory() for _ in range(2)]
+        self.cp_h = [torch.empty((S, 3), dtype=torch.int32).pin_memory() for _ in range(2)]
+        self.h2d_done = [None, None]
+        self.tab_d = torch.empty((S, self.max_blocks), dtype=torch.int32, device=dev)
+        self.len_d = torch.empty((S,), dtype=torch.int32, device=dev)
+        self.pos_d = torch.empty((S,), dtype=torch.int32, device=dev)
+        self.cp_d = torch.empty((S, 3), dtype=torch.int32, device=dev)
+        self.slots = torch.empty((S,), dtype=torch.int64, device=dev)
+        self.ws = pkv.new_workspace(S, Hq, Hkv, D)
+        self.stream = torch.cuda.current_stream()
+        self.parity = 0
+        self.launches = 0
+        self.bytes_done = 0
+        self.attn_bytes = []
+        self.attn_events = []
+        self.record_attn = False
+        # e2e host buffers
+        self.q_h = [self.q[i].cpu().pin_memory() for i in range(L)]
+        self.kn_h = [self.k_new[i].cpu().pin_memory() for i in range(L)]
+        self.vn_h = [self.v_new[i].cpu().pin_memory() for i in range(L)]
+        self.out_h = [torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+
+    def bytes_of_step(self, lens: np.ndarray, n_copies: int) -> int:
+        """Algorithmic bytes: every history slot read once per KV head, q, out, appends, metadata."""
+        e = 2
+        kv = int(lens.sum()) * self.Hkv * self.D * e * 2
+        qo = self.S * self.Hq * self.D * e * 2
+        app = self.S * self.Hkv * self.D * e * 2 * 2
+        meta = 4 * int(sum(-(-int(n) // self.B) for n in lens)) + 4 * self.S
+        cow = n_copies * self.B * self.Hkv * self.D * e * 2 * 2
+        return self.L * (kv + qo + app + meta) + self.L * cow + 8 * self.S
+
+    def attn_bytes_per_launch(self, lens: np.ndarray) -> int:
+        e = 2
+        return (int(lens.sum()) * self.Hkv * self.D * e * 2 + self.S * self.Hq * self.D * e * 2
+                + 4 * int(sum(-(-int(n) // self.B) for n in lens)) + 4 * self.S)
+
+    def step(self, e2e: bool = False):
+        torch, pkv = self.torch, self.pkv
+        rc, nc = self.alloc.append_arrays(self.ids, self.status, self.copies_h)
+        if rc != 0:
+            raise RuntimeError(f"allocator refused a step: {rc}")
+        b = self.parity
+        self.parity ^= 1
+        if self.h2d_done[b] is not None:
+            self.h2d_done[b].synchronize()
+        tab, lens = self.alloc.fill_tables(self.ids, self.max_blocks, 0, self.tab_h[b].numpy(),
+                                           self.len_h[b].numpy())
+        np.subtract(lens, 1, out=self.pos_h[b].numpy())
+        self.tab_d.copy_(self.tab_h[b], non_blocking=True)
+        self.len_d.copy_(self.len_h[b], non_blocking=True)
+        self.pos_d.copy_(self.pos_h[b], non_blocking=True)
+        if nc:
+            self.cp_h[b].numpy()[:nc] = self.copies_h[:nc]
+            self.cp_d[:nc].copy_(self.cp_h[b][:nc], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(self.stream)
+        self.h2d_done[b] = ev
+        if nc:
+            pkv.block_copy(self.k_pools, self.v_pools, self.cp_d[:nc])
+            self.launches += 1
+        pkv.slot_mapping(self.tab_d, self.pos_d, self.B, out=self.slots)
+        pkv.decode_plan(self.len_d, self.Hq, self.Hkv, self.D, pkv.BF16, self.ws)
+        self.launches += 2
+        if e2e:
+            for i in range(self.L):
+                self.q[i].copy_(self.q_h[i], non_blocking=True)
+                self.k_new[i].copy_(self.kn_h[i], non_blocking=True)
+                self.v_new[i].copy_(self.vn_h[i], non_blocking=True)
+        for i in range(self.L):
+            pkv.kv_append(self.k_new[i], self.v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
+            if self.record_attn:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+            pkv.paged_decode_attn_run(self.q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
+                                      self.wl.scale, self.out[i], self.ws)
+            if self.record_attn:
+                e1.record(self.stream)
+                self.attn_events.append((e0, e1))
+                self.attn_bytes.append(self.attn_bytes_per_launch(lens))
+            self.launches += 3
+        if e2e:
+            for i in range(self.L):
+                self.out_h[i].copy_(self.out[i], non_blocking=True)
+        self.bytes_done += self.bytes_of_step(lens, nc)
+
+    def h2d_d2h_bytes(self):
+        e = 2
+        per_layer_in = self.S * self.Hq * self.D * e + 2 * self.S * self.Hkv * self.D * e
+        meta = self.S * self.max_blocks * 4 + self.S * 4
+        return self.L * per_layer_in + meta, self.L * self.S * self.Hq * self.D * e
+
+
+def timed(fn, steps, dist, stream):
+    import torch
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - w0
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    return ms, wall
+
+
+# -- CPU oracle baseline -----------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(seconds: float):
+    """The float64 oracle, as it stands, on a bounded sample of the same workload.
+
+    Requests of the 32 x 4096 batch are drawn and attended one at a time (one
+    layer) until `seconds` of oracle compute have been spent; input generation
+    is not timed.
+    """
+    import workloads as W
+    from oracle import attention as oatt
+
+    wl = W.workload("teaching_32x4096")
+    g = W.rng(123)
+    compute, done_bytes, n_req = 0.0, 0, 0
+    while compute < seconds and n_req < wl.num_seqs:
+        n = wl.lengths[n_req]
+        kh = W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim))
+        vh = W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim))
+        q = W.normal_bf16_bits(g, (wl.num_q_heads, wl.head_dim))
+        t1 = time.perf_counter()
+        oatt.dense_decode(q, kh, vh, wl.scale)
+        compute += time.perf_counter() - t1
+        done_bytes += n * wl.num_kv_heads * wl.head_dim * 2 * 2 + 2 * wl.num_q_heads * wl.head_dim * 2
+        n_req += 1
+    return {"value": done_bytes / compute / 1e9, "unit": "GB/s", "cores": _blas_threads(),
+            "host_cpus": os.cpu_count(), "kind": "oracle",
+            "sample": f"float64 NumPy dense decode attention of {n_req} of the 32 requests x 4096 "
+                      f"history, one layer (H_q 32, H_kv 8, d 128); {compute:.1f} s of CPU work, "
+                      f"input generation not timed"}
+
+
+def reference_arm(args):
+    """--impl reference: the oracle on the host cores, as the comparison arm."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import workloads as W
+    from oracle import attention as oatt
+
+    wl = W.workload("teaching_32x4096")
+    g = W.rng(321)
+    # each step: one layer of a bounded sample (4 requests x 4096 history)
+    reqs = 4
+    hist = [(W.normal_bf16_bits(g, (4096, 8, 128)), W.normal_bf16_bits(g, (4096, 8, 128)),
+             W.normal_bf16_bits(g, (32, 128))) for _ in range(reqs)]
+    step_bytes = reqs * (4096 * 8 * 128 * 2 * 2 + 2 * 32 * 128 * 2)
+
+    def step():
+        for kh, vh, q in hist:
+            oatt.dense_decode(q, kh, vh, wl.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_bytes * args.steps / dt / 1e9
+    threads = _blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1000,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "teaching_32x4096 (bounded sample: 4 of 32 requests, 1 of 32 layers)",
+                       "num_seqs": 32, "history": 4096, "layers": 32, "H_q": 32, "H_kv": 8, "head_dim": 128,
+                       "block_size": 16},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "host_cpus": os.cpu_count(),
+                             "kind": "oracle",
+                             "sample": "each step: float64 NumPy dense decode attention of 4 requests x 4096 "
+                                       "history, one layer"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    import torch
+
+    rank, world, dist = dist_init(args.gpus)
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    budget = 2 * (args.warmup + args.steps) + 4
+    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world)
+    stream = ds.stream
+    for _ in range(args.warmup):
+        ds.step()
+    torch.cuda.synchronize()
+    assert ds.pkv.decode_status(ds.ws) == 0
+
+    # device-resident timed region (with per-launch events on the attention op)
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    ds.bytes_done = 0
+    ds.launches = 0
+    ds.record_attn = True
+    ms, wall = timed(ds.step, args.steps, dist, stream)
+    ds.record_attn = False
+    clk = clocks.stop()
+    launches = ds.launches
+    step_bytes = ds.bytes_done
+    attn_ms = [a.elapsed_time(b) for a, b in ds.attn_events]
+    attn_bytes = ds.attn_bytes
+    assert ds.pkv.decode_status(ds.ws) == 0
+
+    # end-to-end timed region: inputs from pinned host buffers, outputs read back
+    for _ in range(2):
+        ds.step(e2e=True)
+    ds.bytes_done = 0
+    ms_e2e, _ = timed(lambda: ds.step(e2e=True), args.steps, dist, stream)
+    e2e_bytes = ds.bytes_done
+    h2d, d2h = ds.h2d_d2h_bytes()
+
+    ms_max = max_over_ranks(ms, dist)
+    ms_e2e_max = max_over_ranks(ms_e2e, dist)
+    total_bytes = sum_over_ranks(step_bytes, dist)
+    total_e2e = sum_over_ranks(e2e_bytes, dist)
+    value = total_bytes / (ms_max / 1000) / 1e9
+    e2e_value = total_e2e / (ms_e2e_max / 1000) / 1e9
+    peak, peak_kind = peaks()
+    avg_attn_ms = float(np.mean(attn_ms))
+    achieved = float(np.mean(attn_bytes)) / (avg_attn_ms / 1000) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("paged_decode_attn_32x4096_bytes_per_launch")
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(args.cpu_seconds)
+        steps_per_s = args.steps / (ms_max / 1000) * world
+        result = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "teaching_32x4096", "layers": ds.L, "num_seqs": ds.S, "history": 4096,
+                       "H_q": ds.Hq, "H_kv": ds.Hkv, "head_dim": ds.D, "block_size": ds.B,
+                       "pool_blocks_per_layer": ds.N, "kv_pool_gib": round(2 * ds.L * ds.N * ds.B * ds.Hkv * ds.D * 2 / 2**30, 2),
+                       "l2": "inputs larger than L2 (KV pool far above 126 MB); no flush",
+                       "parallelism": f"replicas x{world} (requests sharded by rank, no collective)"},
+            "steps_per_s": steps_per_s, "tokens_per_s": steps_per_s * ds.S,
+            "frac_of_nominal_8tbs": value / NOMINAL_HBM_GBS,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": ms_e2e_max / args.steps},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": "paged_decode_attn (partition + merge), 32x4096 one layer",
+                         "avg_launch_us": avg_attn_ms * 1000,
+                         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS},
+            "cpu_baseline": cpu,
+            "clocks": clk,
+            "gpu_launches": launches,
+            "wall_s_timed": wall,
+        }
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

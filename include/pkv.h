@@ -1,0 +1,315 @@
+/*
+ * pkv.h -- C ABI of libpkv: paged KV-cache decode attention on one NVIDIA B200
+ * (sm_100a), plus the host block allocator that owns the block tables.
+ *
+ * The operations follow three web pages on paged KV caches:
+ *   [P1] "PagedAttention 与在线推理：KV 分页、共享及调度的联合分析"
+ *   [P2] "PagedAttention：让 KV cache 按需生长"
+ *   [P3] "内存预算约束下的语言模型服务：注意力、分页与调度"
+ * Each declaration names the page and section that defines what it computes.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Return value: PKV_OK (0) or one of the PKV_ERR_* codes below.  No C++
+ *   exception crosses this boundary.
+ * - Device pointers are owned by the caller (e.g. allocated by PyTorch) and are
+ *   never freed or retained by the library.  Host pointers are only read or
+ *   written during the call.
+ * - Device calls are asynchronous on the given stream (a cudaStream_t passed
+ *   as void*; NULL is the legacy default stream) and return after the launch.
+ *   Argument checks happen on the host before any launch; a call that returns
+ *   PKV_ERR_INVALID has launched nothing.  PKV_ERR_CUDA means a launch or
+ *   driver call failed; the CUDA error string is available from
+ *   pkv_last_cuda_error().
+ * - Storage types: PKV_BF16 (bfloat16 bit patterns, 2 bytes) or PKV_F32.
+ * - KV pool layout (one K pool and one V pool per layer), the teaching layout
+ *   of [P2] section "把 token 6 变成真正的内存地址":
+ *       pool[num_blocks][block_size][num_kv_heads][head_dim], contiguous.
+ *   Token t of a request lives in logical block t / B at offset t % B; its
+ *   "slot" is block_table[t / B] * B + t % B, the row of the pool viewed as
+ *   [num_blocks * B][num_kv_heads][head_dim] ([P2] sections
+ *   "顺序留在表里，数据放进空闲块" and "读 token 6，先查表，再找偏移").
+ * - Block tables: int32 [num_seqs][max_blocks_per_seq], row s holds the
+ *   physical ids of request s in logical order; entries past
+ *   ceil(seq_lens[s] / B) are never read.
+ * - Supported shapes: head_dim * sizeof(dtype) in {128, 256, 512} bytes
+ *   (bf16: d = 64, 128, 256; f32: d = 32, 64, 128); block_size in
+ *   {1, 2, 4, 8, 16, 32, 64, 128, 256}; num_q_heads % num_kv_heads == 0 with
+ *   group G = num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes -------------------------------------------------------- */
+#define PKV_OK 0
+#define PKV_ERR_NO_BLOCKS 1      /* allocate-or-fail: not enough free blocks      */
+#define PKV_ERR_INVALID 2        /* bad argument, shape, id or range              */
+#define PKV_ERR_CUDA 3           /* a CUDA launch or driver call failed           */
+#define PKV_ERR_DEVICE_TIMEOUT 4 /* a bounded device-side wait ran out            */
+#define PKV_ERR_BAD_TABLE 5      /* a block-table entry was outside [0, blocks)   */
+#define PKV_ERR_PLAN_MISMATCH 6  /* run() with a plan made for other sizes        */
+
+/* storage types */
+#define PKV_BF16 0
+#define PKV_F32 1
+
+typedef void* pkv_stream_t; /* a cudaStream_t */
+
+/* Library version string, e.g. "pkv 0.1.0 sm_100a". */
+const char* pkv_version(void);
+/* Human-readable name of a status code. */
+const char* pkv_status_string(int status);
+/* Text of the last CUDA error seen by this thread (empty if none). */
+const char* pkv_last_cuda_error(void);
+
+/* ==========================================================================
+ * Decode attention
+ * ==========================================================================
+ * What it computes ([P2] section "分页以后，attention 仍然按完整历史归一化";
+ * [P3] section 6 and equation (4)): for every request s and query head h,
+ *     out[s][h] = sum_t softmax_t(scale * <q[s][h], K_t>) V_t,
+ * over the request's tokens t < seq_lens[s], where K_t, V_t are the rows of
+ * KV head h / G found through the block table.  Slots at or past seq_lens[s]
+ * are masked to -inf and never read into a sum (they may hold any bits,
+ * NaN included).  seq_lens[s] == 0 gives out[s] = 0.  The result equals dense
+ * attention over the contiguous history up to floating-point rounding: the
+ * kernels accumulate in fp32 (products of bf16 inputs are exact in fp32).
+ *
+ * How: a persistent split-sequence partition over all (request, KV head,
+ * 16-token tile) units, balanced across every warp of the GPU; each warp keeps
+ * an online-softmax state (m, l, o) for the grouped query heads of one KV
+ * head, reading each K/V tile once per group through a TMA-fed shared-memory
+ * ring; a merge step combines the partial states of requests that were split
+ * ([P2] exercise "逻辑顺序没错，为什么 attention 输出还是错？": the states merge,
+ * per-block outputs do not).
+ *
+ * Arguments (all device pointers unless stated):
+ *   q             [num_seqs][num_q_heads][head_dim], kv_dtype
+ *   k_pool,v_pool [num_blocks][block_size][num_kv_heads][head_dim], kv_dtype;
+ *                 16-byte aligned
+ *   block_tables  int32 [num_seqs][max_blocks_per_seq]
+ *   seq_lens      int32 [num_seqs], 0 <= seq_lens[s] <= max_blocks_per_seq*B
+ *   scale         softmax scale (usually 1/sqrt(head_dim)), host value
+ *   out           [num_seqs][num_q_heads][head_dim], out_dtype (PKV_BF16 rounds
+ *                 the fp32 result to nearest even, PKV_F32 stores it)
+ *   workspace     caller-owned scratch of at least
+ *                 pkv_decode_workspace_bytes(...) bytes, 256-byte aligned; it
+ *                 holds the plan, partial states and a device status word.
+ *                 Calls that share a workspace must be ordered on one stream.
+ * Errors: PKV_ERR_INVALID for unsupported shapes, null or misaligned pointers,
+ * or a workspace that is too small.  Device-detected faults (a block-table
+ * entry outside [0, num_blocks), a bounded wait that ran out) do not stop the
+ * launch: the affected tile reads zeros, and the fault is recorded in the
+ * workspace status word, read back by pkv_decode_status().
+ */
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim);
+
+int pkv_paged_decode_attn(const void* q, const void* k_pool, const void* v_pool,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                          int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                          int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                          int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                          pkv_stream_t stream);
+
+/* The two halves of pkv_paged_decode_attn, for a decode step that runs many
+ * layers over the same seq_lens: plan once, then run once per layer.
+ * pkv_decode_plan reads seq_lens on the device and writes the work partition
+ * into the workspace.  pkv_paged_decode_attn_run uses it; the plan must have
+ * been made with the same num_seqs, num_q_heads, num_kv_heads, head_dim and
+ * kv_dtype on the same seq_lens contents (a mismatch in the sizes is caught on
+ * the device and reported as PKV_ERR_PLAN_MISMATCH by pkv_decode_status()). */
+int pkv_decode_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t kv_dtype, void* workspace,
+                    size_t workspace_bytes, pkv_stream_t stream);
+
+int pkv_paged_decode_attn_run(const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* block_tables, int32_t max_blocks_per_seq,
+                              const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                              int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                              int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                              pkv_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace status word, clears it and
+ * returns PKV_OK, PKV_ERR_BAD_TABLE, PKV_ERR_DEVICE_TIMEOUT or
+ * PKV_ERR_PLAN_MISMATCH (the first recorded), or PKV_ERR_CUDA. */
+int pkv_decode_status(void* workspace, pkv_stream_t stream);
+
+/* Selects the tile kernel for bf16 storage: 0 = automatic (default),
+ * 1 = CUDA-core FMA tiles, 2 = tensor-core (mma.sync bf16) tiles.  fp32
+ * storage always uses FMA tiles.  Process-wide; for measurement. */
+int pkv_set_decode_kernel(int32_t which);
+
+/* ==========================================================================
+ * Cache writes
+ * ==========================================================================
+ * pkv_kv_append -- write the K and V of n_tokens new tokens into their slots
+ * ([P2] section "写满一块，再拿下一块": the new token's K, V go into the tail
+ * block; earlier blocks never move).
+ *   k, v          [n_tokens][num_kv_heads][head_dim], dtype
+ *   slot_mapping  int64 [n_tokens]; pool row = slot (see layout above).  A
+ *                 negative slot (padding) or one >= num_blocks*block_size is
+ *                 skipped.
+ *   k_pool,v_pool one layer's pools
+ * Same-stream ordering makes a preceding pkv_block_copy visible first, as the
+ * allocate-copy-remap-write order of [P2] section
+ * "先确保分配成功，再改变可见状态" requires.
+ */
+int pkv_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t n_tokens,
+                  void* k_pool, void* v_pool, int32_t num_kv_heads, int32_t head_dim,
+                  int32_t block_size, int32_t num_blocks, int32_t dtype, pkv_stream_t stream);
+
+/* pkv_block_copy -- copy-on-write of shared partial tails ([P2] sections
+ * "只读时共用，要写入时再分开" and "一次写入，为什么会先少掉一个空闲块？"):
+ * for each copy i and every layer l,
+ *     pool_l[dst_i][0 : n_valid_i] = pool_l[src_i][0 : n_valid_i]
+ * in both the K and the V pool (block numbering is shared by all layers,
+ * [P2] section "128 KiB：每新增一个位置的账单").
+ *   k_pools,v_pools HOST arrays of num_layers device pool pointers
+ *                   (1 <= num_layers <= 128)
+ *   copies          DEVICE int32 [n_copies][3] = (src, dst, n_valid), the
+ *                   layout pkv_alloc_append() produces; entries with an id
+ *                   outside [0, num_blocks), src == dst, or n_valid outside
+ *                   [0, block_size] are skipped.
+ */
+int pkv_block_copy(void* const* k_pools, void* const* v_pools, int32_t num_layers,
+                   const int32_t* copies, int32_t n_copies, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t dtype,
+                   pkv_stream_t stream);
+
+/* pkv_slot_mapping -- slot of each (request row, position) through the block
+ * table ([P2] sections "读 token 6，先查表，再找偏移" and
+ * "把 token 6 变成真正的内存地址"):
+ *     slots[i] = block_tables[rows[i]][positions[i] / B] * B + positions[i] % B
+ *   rows       DEVICE int32 [n] or NULL (row i for position i)
+ *   positions  DEVICE int32 [n]; a negative position gives slot -1
+ *   slots      DEVICE int64 [n]
+ */
+int pkv_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* rows, const int32_t* positions, int32_t n,
+                     int32_t block_size, int64_t* slots, pkv_stream_t stream);
+
+/* ==========================================================================
+ * Host block allocator
+ * ==========================================================================
+ * Integer metadata only: per request a block table, a length and a state;
+ * per physical block a refcount (number of live requests holding it); a FIFO
+ * free queue; optionally a cached set of released full blocks ([P2] section
+ * "引用计数管理“谁还在读”，长度管理“哪里能写”").  Every call keeps
+ *     active (refcount > 0) + cached + free == num_blocks
+ * ([P2] section "占用率只有 70%，为什么请求还是进不来？").  Every call that returns
+ * an error leaves the allocator exactly as it was, except pkv_alloc_append,
+ * which is all-or-nothing per request (see there).  Not thread-safe: one
+ * thread at a time per handle.  Handles are created and destroyed by the
+ * library.
+ */
+typedef struct pkv_alloc pkv_alloc;
+
+typedef struct pkv_stats {
+  int64_t pool;           /* num_blocks                                   */
+  int64_t active;         /* blocks with refcount > 0                     */
+  int64_t cached;         /* refcount-0 full blocks kept for reuse        */
+  int64_t free;           /* blocks in the free queue                     */
+  int64_t seqs;           /* live requests                                */
+  int64_t allocs;         /* blocks handed out                            */
+  int64_t frees;          /* blocks whose refcount reached 0              */
+  int64_t cow_copies;     /* copy-on-write copies issued                  */
+  int64_t alloc_failures; /* requests refused for lack of blocks          */
+  int64_t evictions;      /* cached blocks reallocated                    */
+} pkv_stats;
+
+/* initial_free_order: host int32 [num_blocks], a permutation of
+ * 0..num_blocks-1 giving the free-queue order (NULL = 0, 1, 2, ...).
+ * enable_cache != 0 keeps released full blocks in the cached set; they are
+ * evicted oldest first, only when the free queue is empty.
+ * Returns NULL on a bad argument or out of host memory. */
+pkv_alloc* pkv_alloc_create(int32_t num_blocks, int32_t block_size,
+                            const int32_t* initial_free_order, int32_t enable_cache);
+void pkv_alloc_destroy(pkv_alloc* a);
+
+/* Admit request seq_id (>= 0, not live) holding n_tokens of KV: takes
+ * ceil(n_tokens / B) blocks from the head of the free queue, or returns
+ * PKV_ERR_NO_BLOCKS and changes nothing ([P2] section
+ * "24 GiB 的 KV 池，能同时容纳多少请求？"). */
+int pkv_alloc_add_seq(pkv_alloc* a, int32_t seq_id, int32_t n_tokens);
+
+/* child (>= 0, not live) shares every block of parent: same table and
+ * length, refcount + 1 on each block ([P2] section "只读时共用，要写入时再分开"). */
+int pkv_alloc_fork(pkv_alloc* a, int32_t parent, int32_t child);
+
+/* Reserve the slot of one new token for each of the n requests, in the given
+ * order ([P2] section "先确保分配成功，再改变可见状态"):
+ *   length % B == 0 (no tail, or tail full)  -> take a free block, append it;
+ *   tail shared (refcount > 1)                -> take a free block, emit the
+ *       copy (tail, new, length % B), refcount[tail] - 1, remap the tail;
+ *   otherwise                                 -> nothing to allocate;
+ * then length + 1.  A request that cannot get its block is left exactly as
+ * it was and its status is PKV_ERR_NO_BLOCKS; later requests still proceed
+ * ([P2] section "三个空闲块，四个请求同时跨边界").
+ *   seq_ids     host int32 [n], live and pairwise distinct, else
+ *               PKV_ERR_INVALID with nothing changed
+ *   status_out  host int32 [n] per-request status
+ *   copies_out  host int32 [n][3] (src, dst, n_valid); *n_copies_out rows used
+ * Returns PKV_OK if every request got its slot, else PKV_ERR_NO_BLOCKS. */
+int pkv_alloc_append(pkv_alloc* a, const int32_t* seq_ids, int32_t n, int32_t* status_out,
+                     int32_t* copies_out, int32_t* n_copies_out);
+
+/* Finish, cancel or preempt: release the request's blocks in logical order;
+ * a block whose refcount reaches 0 goes to the tail of the free queue (or to
+ * the cached set if enabled and it holds B tokens) ([P2] section
+ * "请求结束，块就能交给下一位"). */
+int pkv_alloc_free_seq(pkv_alloc* a, int32_t seq_id);
+
+/* Copy the block table of seq_id into out (host, capacity cap entries);
+ * *len = number of blocks, *n_tokens = its length.  PKV_ERR_INVALID if the
+ * request is not live or cap is too small. */
+int pkv_alloc_get_table(const pkv_alloc* a, int32_t seq_id, int32_t* out, int32_t cap,
+                        int32_t* len, int32_t* n_tokens);
+
+/* Fill host tables_out [n][max_blocks_per_seq] (row i = request seq_ids[i],
+ * unused entries = pad) and host seq_lens_out [n], ready to mirror to the
+ * device.  PKV_ERR_INVALID if a request is not live or its table is longer
+ * than max_blocks_per_seq (nothing written then). */
+int pkv_alloc_fill_tables(const pkv_alloc* a, const int32_t* seq_ids, int32_t n,
+                          int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
+                          int32_t* seq_lens_out);
+
+int pkv_alloc_stats(const pkv_alloc* a, pkv_stats* out);
+
+/* Full consistency check: conservation, a refcount recount from the live
+ * tables, table lengths, no block both idle and referenced.  PKV_OK or
+ * PKV_ERR_INVALID. */
+int pkv_alloc_check(const pkv_alloc* a);
+
+/* Snapshot for tests: refcounts [num_blocks], the free queue and the cached
+ * set in order (host arrays of capacity num_blocks; counts written to
+ * *n_free, *n_cached).  Any pointer may be NULL to skip that part. */
+int pkv_alloc_dump(const pkv_alloc* a, int32_t* refcounts, int32_t* free_order, int32_t* n_free,
+                   int32_t* cached_order, int32_t* n_cached);
+
+/* Host-side fault injection for failure tests (no device involvement):
+ *   PKV_FAULT_ALLOC_FAIL    the next `count` block allocations fail as if
+ *                           the pool were empty;
+ *   PKV_FAULT_SKIP_RELEASE  the next `count` pkv_alloc_free_seq calls drop the
+ *                           request without releasing its references (a leak
+ *                           that pkv_alloc_check reports);
+ *   PKV_FAULT_NONE          clears pending faults. */
+#define PKV_FAULT_NONE 0
+#define PKV_FAULT_ALLOC_FAIL 1
+#define PKV_FAULT_SKIP_RELEASE 2
+int pkv_alloc_inject_fault(pkv_alloc* a, int32_t kind, int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,108 @@
+// Shared pieces of the decode-attention kernels: workspace layout, the
+// per-warp stream-K worker (its TMA ring, block-table lookahead and pair
+// bookkeeping) and the tile-core interface the FMA and MMA cores implement.
+//
+// The method is PagedAttention decode as "PagedAttention：让 KV cache 按需生长"
+// (hs-black.github.io) states it in section
+// "分页以后，attention 仍然按完整历史归一化": for each logical block look up the
+// physical block, load its K/V tile, mask slots at or past the length, score
+// q K^T * scale and apply the online-softmax update; equation (4) of
+// "内存预算约束下的语言模型服务：注意力、分页与调度" gives the update
+//   m' = max(m, max_j s_j),  l' = e^{m-m'} l + sum_j e^{s_j-m'},
+// with the value accumulator rescaled by e^{m-m'}.  Scores are kept in the
+// log2 domain (q is pre-multiplied by scale * log2(e)), so every e^x becomes
+// 2^x on the same exponent: the same function, one multiply fewer per score.
+//
+// Work decomposition (our design, not the pages'): a "pair" is (request s,
+// KV head g); a pair's history is cut into 16-token tiles.  All tiles of all
+// pairs form one flattened sequence ordered (s, g, tile), which is split into
+// equal contiguous ranges, one per warp of a persistent grid (a warp-level
+// stream-K).  Each warp walks its range with a private ring of shared-memory
+// stages fed by TMA (cp.async.bulk.tensor), so a long request is spread over
+// many warps and short ones pack together; every warp gets the same number of
+// tiles (+-1) whatever the length mix.  A warp keeps one (m, l, o) state per
+// grouped query head; when its range covers a whole pair it writes the final
+// output, otherwise it writes a partial state that the merge kernel combines.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int kTile = 16;          // tokens per tile
+constexpr int kMaxBoxes = 4;       // TMA boxes per tile (block_size >= 4)
+constexpr int kBatch = 32;         // tiles of table lookahead per warp
+
+struct WsHeader {
+  uint32_t status;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t kv_dtype;
+  int32_t num_workers;
+  int32_t planned;
+  long long total_tiles;
+};
+
+// Workspace layout (byte offsets, each 256-aligned):
+//   header | prefix int32[S+1] (tiles per request, cumulative) |
+//   worker plan int4[NW] {tile_begin, tile_end, s, offset in s} |
+//   partial states float[NW + S*H_kv][part_stride(G, D)]  (o[G][D], m[G], l[G],
+//   padded so every slot starts on a 16-byte boundary)
+constexpr int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
+
+struct WsLayout {
+  size_t prefix = 0, wplan = 0, partials = 0, total = 0;
+  WsLayout() = default;
+  static size_t up(size_t x) { return (x + 255) & ~size_t(255); }
+  WsLayout(int S, int H_kv, int G, int D, int NW) {
+    prefix = up(sizeof(WsHeader));
+    wplan = prefix + up(sizeof(int32_t) * (size_t(S) + 1));
+    partials = wplan + up(sizeof(int4) * size_t(NW));
+    total = partials + up(sizeof(float) * (size_t(NW) + size_t(S) * H_kv) * part_stride(G, D));
+  }
+};
+
+struct DecodeArgs {
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  void* out;
+  char* ws;
+  size_t off_prefix, off_wplan, off_partials;
+  int32_t max_blocks;   // table row stride
+  int32_t num_seqs, num_q_heads, num_kv_heads;
+  int32_t block_size, num_blocks;
+  int32_t out_dtype;
+  int32_t num_workers;
+  float scale_log2;     // scale * log2(e)
+};
+
+PKV_DEVINL void store1(void* out, int out_dtype, size_t off, float v) {
+  if (out_dtype == 1)
+    reinterpret_cast<float*>(out)[off] = v;
+  else
+    reinterpret_cast<__nv_bfloat16*>(out)[off] = __float2bfloat16_rn(v);
+}
+
+PKV_DEVINL int ntiles_of(int len) { return len > 0 ? (len + kTile - 1) / kTile : 0; }
+
+// Worker that owns flattened tile t when T tiles are split over NW workers
+// (worker v owns [floor(v T / NW), floor((v+1) T / NW))).
+PKV_DEVINL int owner_of(long long t, long long T, int NW) {
+  return static_cast<int>(((t + 1) * NW - 1) / T);
+}
+PKV_DEVINL long long range_begin(int v, long long T, int NW) {
+  return (static_cast<long long>(v) * T) / NW;
+}
+
+// Per-stage metadata written by the issuing lane, read by the consuming warp.
+struct StageMeta {
+  int32_t s;       // request
+  int32_t g;       // KV head
+  int32_t j;       // tile index within the pair
+  int32_t flags;   // bit 0: first tile of a pair in this warp (q staged); bits 8..: nvalid
+};
+
+}  // namespace pkv

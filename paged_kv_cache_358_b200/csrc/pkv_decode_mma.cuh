@@ -1,0 +1,249 @@
+// Tensor-core tile core of the decode kernel for bf16 pools (mma.sync
+// m16n8k16, bf16 inputs, fp32 accumulation).
+//
+// Decode attention is a streaming read with G flops per byte (G = grouped
+// query heads per KV head), far below any tensor-core ridge; the tensor cores
+// here only take the multiply-adds off the CUDA cores, whose issue slots
+// would otherwise bound the kernel below HBM speed at G = 4..8.  tcgen05 needs
+// M >= 64 and a TMEM round trip per tile for the softmax; the warp-level
+// m16n8k16 shape fits one 16-token tile and the grouped heads directly.
+//
+// Shapes per 16-token tile (tokens in M, grouped heads in N padded to 8):
+//   scores  S^T[16 tok x 8 heads] = K[16 x D] * Q^T[D x 8]      (D/16 MMAs)
+//   values  O^T[D x 8 heads]     += V^T[D x 16 tok] * P^T[16 x 8] (D/16 MMAs)
+// K and V tiles arrive through TMA with the 128-byte swizzle, so ldmatrix
+// (plain for K, .trans for V^T) reads them without bank conflicts.  The
+// score accumulator (token-major) is turned into the P^T operand of the value
+// MMA with movmatrix.trans, after the online-softmax update of [P3] eq. (4)
+// in fp32 on the accumulator registers.  P is rounded to bf16 for the value
+// MMA (relative error <= 2^-9 per weight); everything else stays fp32.
+// Slots at or past the length: their scores are replaced by -inf, and in the
+// last tile their V^T operand columns are zeroed before the MMA, so stale NaN
+// rows cannot reach the accumulator through 0 * NaN.
+#pragma once
+
+#include "pkv_decode_fma.cuh"
+
+namespace pkv {
+
+PKV_DEVINL void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+PKV_DEVINL void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+PKV_DEVINL void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+PKV_DEVINL uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+PKV_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D, int G>
+struct MmaCore {
+  static constexpr int ESZ = 2;
+  static constexpr int ROWB = D * ESZ;
+  static constexpr int NCH = ROWB / 128;      // 128-byte swizzle atoms per row
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int CHUNKB = kTile * 128;  // one swizzled chunk of a tile
+  static constexpr int TILEB = NCH * CHUNKB;
+  static constexpr int QB = G * ROWB;
+  static constexpr int kAlign = 1024;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = TILEB;
+  static constexpr int kQOff = 2 * TILEB;
+  static constexpr int kStageBytes = round_up(2 * TILEB + QB, 1024);
+  static constexpr int kChunks = NCH;
+  static constexpr int kBoxInner = 64;  // bf16 elements per 128-byte box row
+  static constexpr int kChunkRowBytes = 128;
+  static constexpr int kChunkBytes = CHUNKB;
+  static constexpr bool kSwizzle = true;
+  static constexpr int kScratchBytes = 0;
+
+  static_assert(G >= 1 && G <= 8, "grouped heads must fit the 8 MMA columns");
+  static_assert(NCH >= 1 && NCH <= 4, "head_dim 64, 128 or 256");
+
+  struct State {
+    uint32_t qb[KSTEPS][2];  // Q^T B-fragments (bf16x2), heads >= G are zero
+    float oc[KSTEPS][4];     // O^T accumulator: rows d = 16*mt + gid (+8), cols heads 2*tig (+1)
+    float m[2];              // running max of heads 2*tig, 2*tig+1 (log2 domain)
+    float l[2];              // this lane's share of the running sums
+  };
+
+  // Byte offset of (row t, 16-byte unit) inside a swizzled tile.
+  static PKV_DEVINL uint32_t swz(int t, int unit) {
+    return static_cast<uint32_t>((unit >> 3) * CHUNKB + t * 128 + (((unit & 7) ^ (t & 7)) << 4));
+  }
+
+  static PKV_DEVINL void begin_pair(State& st, const char* qsm, float /*scale_log2*/, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      if (gid < G) {
+        const char* row = qsm + gid * ROWB + (16 * kk + 2 * tig) * 2;
+        st.qb[kk][0] = *reinterpret_cast<const uint32_t*>(row);
+        st.qb[kk][1] = *reinterpret_cast<const uint32_t*>(row + 16);
+      } else {
+        st.qb[kk][0] = 0u;
+        st.qb[kk][1] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.oc[kk][i] = 0.f;
+    }
+    st.m[0] = st.m[1] = -INFINITY;
+    st.l[0] = st.l[1] = 0.f;
+  }
+
+  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, int nvalid, float scale_log2,
+                              int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
+
+    // scores S^T = K Q^T
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int t = lane & 15;
+      const int cb = lane >> 4;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kbase + swz(t, 2 * kk + cb), a0, a1, a2, a3);
+        mma_bf16_16816(c, a0, a1, a2, a3, st.qb[kk][0], st.qb[kk][1]);
+      }
+    }
+    // c[0]: (tok gid, head 2tig), c[1]: (gid, 2tig+1), c[2]: (gid+8, 2tig), c[3]: (gid+8, 2tig+1)
+    float s[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = gid + ((i & 2) ? 8 : 0);
+      s[i] = t < nvalid ? c[i] * scale_log2 : -INFINITY;
+    }
+    float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+    for (int msk = 4; msk < 32; msk <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+    }
+    const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+    const float al0 = exp2f(st.m[0] - mn0), al1 = exp2f(st.m[1] - mn1);
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+    const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
+    const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
+    st.l[0] = st.l[0] * al0 + (p0 + p2);
+    st.l[1] = st.l[1] * al1 + (p1 + p3);
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        st.oc[mt][0] *= al0;
+        st.oc[mt][1] *= al1;
+        st.oc[mt][2] *= al0;
+        st.oc[mt][3] *= al1;
+      }
+    }
+    // P^T operand: transpose the token-major fragments
+    const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
+
+    // values O^T += V^T P^T
+    const int vt = ((lane >> 4) << 3) + (lane & 7);
+    const int vu = (lane >> 3) & 1;
+    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+    const bool tail = nvalid < kTile;
+    if (tail) {
+      mlo = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+      mhi = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(vbase + swz(vt, 2 * mt + vu), a0, a1, a2, a3);
+      if (tail) {
+        a0 &= mlo;
+        a1 &= mlo;
+        a2 &= mhi;
+        a3 &= mhi;
+      }
+      mma_bf16_16816(st.oc[mt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+  static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, size_t out_row,
+                                float* part, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    float l0 = st.l[0], l1 = st.l[1];
+#pragma unroll
+    for (int msk = 4; msk < 32; msk <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
+    }
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+    if (complete) {
+      const float i0 = 1.f / l0, i1 = 1.f / l1;
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        if (h0 < G) {
+          put(out, out_dtype, out_row + size_t(h0) * D + d0, st.oc[mt][0] * i0);
+          put(out, out_dtype, out_row + size_t(h0) * D + d1, st.oc[mt][2] * i0);
+        }
+        if (h1 < G) {
+          put(out, out_dtype, out_row + size_t(h1) * D + d0, st.oc[mt][1] * i1);
+          put(out, out_dtype, out_row + size_t(h1) * D + d1, st.oc[mt][3] * i1);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        if (h0 < G) {
+          part[h0 * D + d0] = st.oc[mt][0];
+          part[h0 * D + d1] = st.oc[mt][2];
+        }
+        if (h1 < G) {
+          part[h1 * D + d0] = st.oc[mt][1];
+          part[h1 * D + d1] = st.oc[mt][3];
+        }
+      }
+      if (gid == 0) {
+        if (h0 < G) {
+          part[G * D + h0] = st.m[0];
+          part[G * D + G + h0] = l0;
+        }
+        if (h1 < G) {
+          part[G * D + h1] = st.m[1];
+          part[G * D + G + h1] = l1;
+        }
+      }
+    }
+  }
+
+  static PKV_DEVINL void put(void* out, int out_dtype, size_t off, float v) {
+    if (out_dtype == 1)
+      reinterpret_cast<float*>(out)[off] = v;
+    else
+      reinterpret_cast<__nv_bfloat16*>(out)[off] = __float2bfloat16_rn(v);
+  }
+};
+
+}  // namespace pkv

@@ -1,0 +1,360 @@
+"""Paged decode attention on the GPU against the float64 oracle.
+
+Tolerances (max |out - oracle|):
+  * fp32 pools, fp32 accumulation: 1e-5;
+  * bf16 pools, fp32 accumulation: 1e-2 for an fp32 output; a bf16 output
+    adds half a bf16 ulp of the value (its final rounding, 2^-8 |x|).
+Small cases compare every output; the full-size workloads compare sampled
+(request, head) outputs that the oracle computes one by one, plus properties
+that hold at any size (finite outputs, length-1 requests return v_0).
+Pools are filled with NaN before the history is written, so any read of a slot
+at or past a request's length shows up in the output.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from tests.paged_batch import as_f64, bf16_out_tol, device_batch, host_batch, oracle_out
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-2
+
+
+@pytest.fixture(params=[0, 1, 2], ids=["auto", "fma", "mma"])
+def kernel(request):
+    import paged_kv_cache_358_b200 as pkv
+
+    pkv.set_decode_kernel(request.param)
+    yield request.param
+    pkv.set_decode_kernel(0)
+
+
+def _run(db, hb, out_dtype):
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    ws = pkv.new_workspace(len(hb.lengths), hb.wl.num_q_heads, hb.wl.num_kv_heads, hb.wl.head_dim)
+    out = pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, hb.wl.scale,
+                                out_dtype=out_dtype, workspace=ws)
+    assert pkv.decode_status(ws) == 0
+    torch.cuda.synchronize()
+    return out
+
+
+def _check(got, ref, out_is_bf16, base):
+    tol = bf16_out_tol(ref, base) if out_is_bf16 else base
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got))
+    assert np.all(err <= tol), f"max err {err.max():.3e} (tol {np.max(tol):.3e})"
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_edge"])
+def test_tiny_fp32_all_outputs(name):
+    """Lengths 37/91/128/201/511 and the edge batch 0/1/16/17, fp32, B = 16."""
+    import torch
+
+    wl = W.workload(name)
+    hb = host_batch(wl)
+    db = device_batch(hb)
+    ref = oracle_out(hb)
+    for od in (torch.float32, torch.bfloat16):
+        got = as_f64(_run(db, hb, od))
+        _check(got, ref, od == torch.bfloat16, TOL_F32)
+    if name == "tiny_edge":
+        got = as_f64(_run(db, hb, torch.float32))
+        assert np.array_equal(got[0], np.zeros_like(got[0]))          # length 0 gives 0
+        assert np.array_equal(got[1], ref[1])                          # length 1 gives v_0 exactly
+
+
+def test_tiny_nine_requests_in_one_pool_fail_cleanly():
+    """All nine tiny requests need 66 blocks of a 64-block pool: the one that overflows is refused."""
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("tiny")
+    a = pkv.BlockAllocator(64, 16)
+    results = [a.add_seq(i, n) for i, n in enumerate([37, 91, 128, 201, 511, 0, 1, 16, 17])]
+    assert results[:8] == [0] * 8 and results[8] == pkv.Status.NO_BLOCKS
+    assert a.stats()["free"] == 64 - 64 and a.check()
+    assert wl.pool_blocks == 64
+
+
+@pytest.mark.parametrize("B", [4, 8, 16, 32, 64])
+@pytest.mark.parametrize("G,Hkv,D", [(4, 8, 128), (8, 4, 128), (1, 4, 64), (2, 2, 64), (4, 2, 256)])
+def test_bf16_mixed_lengths(kernel, B, G, Hkv, D):
+    import torch
+
+    lengths = [0, 1, B, B + 1, 15, 16, 17, 33, 100, 257, 513, 1000]
+    base = W.workload("mixed_512", block_size=B)
+    wl = W.DecodeWorkload("mixed", 1, G * Hkv, Hkv, D, B, "bf16", lengths,
+                          pool_blocks=sum(-(-n // B) for n in lengths) + 7, seed=11 + B)
+    hb = host_batch(wl)
+    db = device_batch(hb)
+    ref = oracle_out(hb)
+    for od in (torch.float32, torch.bfloat16):
+        got = as_f64(_run(db, hb, od))
+        _check(got, ref, od == torch.bfloat16, TOL_BF16)
+    assert base.block_size == B
+
+
+@pytest.mark.parametrize("B", [4, 8, 16, 32, 64])
+def test_mixed_512_block_sweep(kernel, B):
+    """512 requests, lengths uniform on 1..512, H_q 32 / H_kv 8 / d 128, every output."""
+    import torch
+
+    wl = W.workload("mixed_512", block_size=B)
+    hb = host_batch(wl)
+    db = device_batch(hb)
+    ref = oracle_out(hb)
+    got = as_f64(_run(db, hb, torch.float32))
+    _check(got, ref, False, TOL_BF16)
+
+
+@pytest.mark.parametrize("qscale", [30.0, 1000.0])
+def test_extreme_logits(kernel, qscale):
+    """q scaled x30 and x1000 (|s| ~ 1e3): the running max keeps every exponent finite."""
+    import torch
+
+    wl = W.workload("mixed_512", block_size=16)
+    hb = host_batch(wl, q_scale=qscale)
+    db = device_batch(hb)
+    ref = oracle_out(hb)
+    for od in (torch.float32, torch.bfloat16):
+        got = as_f64(_run(db, hb, od))
+        _check(got, ref, od == torch.bfloat16, TOL_BF16)
+
+
+def test_permutation_invariance():
+    """The same histories behind two different physical block orders give the same output."""
+    import torch
+
+    wl = W.workload("mixed_512", block_size=16)
+    lengths = list(wl.lengths)[:96]
+    hb1 = host_batch(wl, lengths=lengths)
+    hb2 = host_batch(wl, lengths=lengths)
+    hb2.order = np.ascontiguousarray(hb1.order[::-1])
+    o1 = _run(device_batch(hb1), hb1, torch.float32)
+    o2 = _run(device_batch(hb2), hb2, torch.float32)
+    assert torch.equal(o1, o2)
+
+
+_CACHE = {}
+
+
+def _cached(name):
+    """Full-size batches are built once per module and shared by the kernel variants."""
+    if name not in _CACHE:
+        _CACHE.clear()
+        hb = host_batch(W.workload(name))
+        _CACHE[name] = (hb, device_batch(hb))
+    return _CACHE[name]
+
+
+def _sampled(hb, got, n=48, seed=5):
+    g = W.rng(seed)
+    S, H = got.shape[0], got.shape[1]
+    rows = [(int(g.integers(0, S)), int(g.integers(0, H))) for _ in range(n)]
+    ref = oracle_out(hb, rows=rows)
+    return np.stack([got[s, h] for s, h in rows]), ref
+
+
+def test_teaching_32x4096_one_layer_sampled(kernel):
+    """32 requests x 4096 history, H_q 32 / H_kv 8 / d 128, bf16, B 16 (one layer)."""
+    import torch
+
+    hb, db = _cached("teaching_32x4096")
+    got = as_f64(_run(db, hb, torch.bfloat16))
+    assert np.all(np.isfinite(got))
+    g, r = _sampled(hb, got)
+    _check(g, r, True, TOL_BF16)
+
+
+def test_large_serving_gqa8_sampled(kernel):
+    """256 requests, lengths uniform on 1..8192, H_q 32 / H_kv 4 (G = 8), bf16, B 16."""
+    import torch
+
+    hb, db = _cached("large_serving")
+    wl = hb.wl
+    got = as_f64(_run(db, hb, torch.float32))
+    assert np.all(np.isfinite(got))
+    g, r = _sampled(hb, got, n=64)
+    _check(g, r, False, TOL_BF16)
+    # property at full size: every length-1 request returns its single v
+    for s, n in enumerate(hb.lengths):
+        if n == 1:
+            vf = as_f64(db.v_pool[int(db.tables[s, 0]), 0])
+            for h in range(wl.num_q_heads):
+                assert np.max(np.abs(got[s, h] - vf[h // wl.group])) <= 1e-6
+
+
+def test_prefix_sharing_with_cow():
+    """Groups of 4 branches share a 2008-token prompt (shared 8-slot tail), each appends 3 tokens.
+
+    Three branches of every group copy the tail (block_copy), the last writes in
+    place; attention of every branch equals dense attention over prompt + its
+    own tokens."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    from oracle import attention as oatt
+    from oracle.allocator import RefAllocator
+
+    wl = W.workload("prefix_cow")
+    groups, branches, prompt, steps = 8, 4, 2008, 3
+    B, Hkv, D, Hq = wl.block_size, wl.num_kv_heads, wl.head_dim, wl.num_q_heads
+    g = W.rng(wl.seed)
+    N = groups * (-(-prompt // B) + branches * 2) + 8
+    order = W.free_order(g, N)
+    a = pkv.BlockAllocator(N, B, free_order=order)
+    r = RefAllocator(N, B, free_order=order)
+    sids = []
+    prompts_k = [W.normal_bf16_bits(g, (prompt, Hkv, D)) for _ in range(groups)]
+    prompts_v = [W.normal_bf16_bits(g, (prompt, Hkv, D)) for _ in range(groups)]
+    kp = torch.full((N, B, Hkv, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vp = torch.full_like(kp, float("nan"))
+    for gi in range(groups):
+        root = gi * branches
+        assert a.add_seq(root, prompt) == 0 and r.add_seq(root, prompt) == 0
+        for b in range(1, branches):
+            assert a.fork(root, root + b) == 0 and r.fork(root, root + b) == 0
+        sids += [root + b for b in range(branches)]
+        t = torch.tensor([a.table(root)], dtype=torch.int32, device="cuda")
+        slots = pkv.slot_mapping(t, torch.arange(prompt, dtype=torch.int32, device="cuda"), B,
+                                 rows=torch.zeros(prompt, dtype=torch.int32, device="cuda"))
+        pkv.kv_append(torch.from_numpy(prompts_k[gi].view(np.int16)).view(torch.bfloat16).cuda(),
+                      torch.from_numpy(prompts_v[gi].view(np.int16)).view(torch.bfloat16).cuda(), slots, kp, vp)
+    new_k = {s: [] for s in sids}
+    new_v = {s: [] for s in sids}
+    maxb = -(-(prompt + steps) // B)
+    total_copies = 0
+    for step in range(steps):
+        rc, per, copies = a.append(sids)
+        assert (rc, per, copies) == r.append(sids) and rc == 0
+        total_copies += len(copies)
+        if copies:
+            pkv.block_copy([kp], [vp], torch.tensor(copies, dtype=torch.int32, device="cuda"))
+        tables, lens = a.fill_tables(sids, maxb)
+        td = torch.from_numpy(tables).cuda()
+        slots = pkv.slot_mapping(td, torch.from_numpy(lens - 1).cuda(), B)
+        kn = W.normal_bf16_bits(g, (len(sids), Hkv, D))
+        vn = W.normal_bf16_bits(g, (len(sids), Hkv, D))
+        for i, s in enumerate(sids):
+            new_k[s].append(kn[i])
+            new_v[s].append(vn[i])
+        pkv.kv_append(torch.from_numpy(kn.view(np.int16)).view(torch.bfloat16).cuda(),
+                      torch.from_numpy(vn.view(np.int16)).view(torch.bfloat16).cuda(), slots, kp, vp)
+    assert total_copies == groups * (branches - 1)          # first step only, in-place for the last holder
+    assert a.check() and r.check()
+    q = W.normal_bf16_bits(g, (len(sids), Hq, D))
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).cuda()
+    tables, lens = a.fill_tables(sids, maxb)
+    out = pkv.paged_decode_attn(qd, kp, vp, torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(),
+                                wl.scale, out_dtype=torch.float32)
+    got = as_f64(out)
+    for i, s in enumerate(sids):
+        gi = s // branches
+        kh = np.concatenate([prompts_k[gi], np.stack(new_k[s])])
+        vh = np.concatenate([prompts_v[gi], np.stack(new_v[s])])
+        ref = oatt.dense_decode(q[i], kh, vh, wl.scale)
+        assert np.max(np.abs(got[i] - ref)) <= TOL_BF16
+
+
+def test_plan_once_run_per_layer():
+    """pkv_decode_plan + run on two layers equals the one-shot call on each."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("mixed_512", block_size=16)
+    lengths = list(wl.lengths)[:200]
+    hb = host_batch(wl, lengths=lengths)
+    d1 = device_batch(hb)
+    d2 = device_batch(hb)
+    d2.k_pool.copy_(d1.v_pool)
+    d2.v_pool.copy_(d1.k_pool)
+    ws = pkv.new_workspace(len(lengths), wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+    pkv.decode_plan(d1.seq_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, pkv.BF16, ws)
+    outs = []
+    for db in (d1, d2):
+        o = torch.empty(d1.q.shape, dtype=torch.float32, device="cuda")
+        pkv.paged_decode_attn_run(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale, o, ws)
+        outs.append(o)
+    for db, o in zip((d1, d2), outs):
+        ref = pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale,
+                                    out_dtype=torch.float32)
+        assert torch.equal(o, ref)
+    assert pkv.decode_status(ws) == 0
+
+
+def test_plan_mismatch_is_reported():
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("mixed_512", block_size=16)
+    hb = host_batch(wl, lengths=list(wl.lengths)[:40])
+    db = device_batch(hb)
+    ws = pkv.new_workspace(64, wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+    pkv.decode_plan(db.seq_lens[:30], wl.num_q_heads, wl.num_kv_heads, wl.head_dim, pkv.BF16, ws)
+    o = torch.zeros(db.q.shape, dtype=torch.float32, device="cuda")
+    pkv.paged_decode_attn_run(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale, o, ws)
+    assert pkv.decode_status(ws) == pkv.Status.PLAN_MISMATCH
+    assert pkv.decode_status(ws) == 0          # read clears it
+
+
+def test_bad_table_entry_is_reported_and_reads_zeros():
+    """A physical id outside the pool is flagged; its tile reads zeros (TMA bounds), nothing faults."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("mixed_512", block_size=16)
+    hb = host_batch(wl, lengths=[40, 40])
+    db = device_batch(hb)
+    db.tables[1, 1] = wl.pool_blocks + 5
+    ws = pkv.new_workspace(2, wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+    out = pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale,
+                                out_dtype=torch.float32, workspace=ws)
+    assert pkv.decode_status(ws) == pkv.Status.BAD_TABLE
+    ref = oracle_out(hb)
+    assert np.max(np.abs(as_f64(out)[0] - ref[0])) <= TOL_BF16      # the other request is unaffected
+    assert np.all(np.isfinite(as_f64(out)))
+
+
+def test_invalid_arguments_launch_nothing():
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("mixed_512", block_size=16)
+    hb = host_batch(wl, lengths=[10, 20])
+    db = device_batch(hb)
+    small = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale, workspace=small)
+    assert e.value.status == pkv.Status.INVALID
+    L = pkv.lib()
+    ws = pkv.new_workspace(2, 32, 8, 128)
+    for Hq, Hkv, D, B in ((32, 8, 96, 16), (30, 8, 128, 16), (32, 8, 128, 12), (96, 4, 128, 16)):
+        rc = L.pkv_paged_decode_attn(db.q.data_ptr(), db.k_pool.data_ptr(), db.v_pool.data_ptr(),
+                                     db.tables.data_ptr(), db.max_blocks, db.seq_lens.data_ptr(), 2, Hq, Hkv,
+                                     D, B, wl.pool_blocks, 0.1, pkv.BF16, db.q.data_ptr(), pkv.BF16,
+                                     ws.data_ptr(), ws.numel(), None)
+        assert rc == pkv.Status.INVALID
+
+
+def test_empty_batch_and_all_zero_lengths():
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    wl = W.workload("mixed_512", block_size=16)
+    hb = host_batch(wl, lengths=[0, 0, 0])
+    db = device_batch(hb)
+    out = torch.full(db.q.shape, 7.0, dtype=torch.float32, device="cuda")
+    pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale, out=out)
+    assert torch.count_nonzero(out) == 0
+    e = pkv.paged_decode_attn(db.q[:0], db.k_pool, db.v_pool, db.tables[:0], db.seq_lens[:0], wl.scale)
+    assert e.shape[0] == 0
