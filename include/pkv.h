@@ -139,6 +139,29 @@ int pkv_paged_decode_attn_run(const void* q, const void* k_pool, const void* v_p
                               int32_t out_dtype, void* workspace, size_t workspace_bytes,
                               pkv_stream_t stream);
 
+/* Allocation-free variant of pkv_paged_decode_attn (the pages have no
+ * counterpart: this is a deployment convenience).  For callers that cannot
+ * allocate device memory -- e.g. a plugin called by a runtime that owns all
+ * device allocations and passes only inputs and outputs, or a serving loop
+ * that must never call cudaMalloc -- the scratch lives in a 16 MiB array
+ * built into the library (held on every GPU that loads it, until exit).
+ * Arguments are those of pkv_paged_decode_attn without the workspace.
+ * - Batches whose pkv_decode_workspace_bytes() exceeds 16 MiB are refused
+ *   with PKV_ERR_INVALID (pkv_last_cuda_error() says why); nothing runs.
+ * - The first call on each device looks up the array's device address; make
+ *   that first call before any stream capture.
+ * - No call allocates: no cudaMalloc/cudaFree, no allocating library routine.
+ * - All calls share the one array per device: calls that overlap on the GPU
+ *   (different streams without ordering) race and give wrong results.  Each
+ *   call clears the status word it uses; device-detected faults are not
+ *   reported back (use the workspace form when they must be). */
+int pkv_paged_decode_attn_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                                  int32_t out_dtype, pkv_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace status word, clears it and
  * returns PKV_OK, PKV_ERR_BAD_TABLE, PKV_ERR_DEVICE_TIMEOUT or
  * PKV_ERR_PLAN_MISMATCH (the first recorded), or PKV_ERR_CUDA. */

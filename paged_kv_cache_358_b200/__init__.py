@@ -74,6 +74,8 @@ _SIGS = {
     "pkv_paged_decode_attn_run": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                  _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "pkv_decode_status": (ctypes.c_int, [_vp, _vp]),
+    "pkv_paged_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                                                     _i32, _i32, _f32, _i32, _vp, _i32, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
     "pkv_kv_append": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_block_copy": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _vp, _i32, _i32, _i32,

@@ -685,3 +685,68 @@ int pkv_set_decode_kernel(int32_t which) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free decode attention
+// ===========================================================================
+// Some callers cannot hand us device scratch: a plugin invoked by a host
+// runtime that owns every device allocation and passes a kernel only its
+// inputs and outputs, or a latency-critical serving loop that must never call
+// cudaMalloc (it synchronises the device and can fail late under memory
+// pressure).  For them the entry point below keeps its scratch in a
+// fixed-size array that lives in this library's device image: every GPU that
+// loads the library holds these bytes until the process exits, and no call
+// allocates anything.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device.  The array's
+// name is only a host-side stand-in in host code, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return host::cuda_fail(e);
+  if (dev < 0 || dev >= 64) return PKV_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return host::cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_decode_attn_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* seq_lens, int32_t num_seqs,
+                                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                             int32_t block_size, int32_t num_blocks, float scale,
+                                             int32_t kv_dtype, void* out, int32_t out_dtype,
+                                             pkv_stream_t stream) {
+  Geometry geo;
+  if (!geometry(num_seqs, num_q_heads, num_kv_heads, head_dim, kv_dtype, &geo)) return PKV_ERR_INVALID;
+  if (geo.lay.total > kNoAllocScratchBytes) {
+    host::set_error("decode batch needs more scratch than the 16 MiB built into the library");
+    return PKV_ERR_INVALID;
+  }
+  void* ws = nullptr;
+  int rc = noalloc_scratch(&ws);
+  if (rc != PKV_OK) return rc;
+  // The array keeps the previous call's contents: clear the header (status
+  // word and plan marker) before this call plans into it.
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return host::cuda_fail(e);
+  return pkv_paged_decode_attn(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                               num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype,
+                               out, out_dtype, ws, kNoAllocScratchBytes, stream);
+}
