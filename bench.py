@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
+    p.add_argument("--layers", type=int, default=32,
+                   help="layers per step (32 for the workload; fewer only for small profiling captures)")
     return p.parse_args()
 
 
@@ -171,7 +173,8 @@ class ClockSampler:
 class DecodeStep:
     """32-layer decode step through the C ABI; all state resident on the device."""
 
-    def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1):
+    def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1,
+                 layers: int = 32):
         import torch
 
         import paged_kv_cache_358_b200 as pkv
@@ -181,7 +184,7 @@ class DecodeStep:
         pkv.set_decode_kernel(kernel)
         wl = W.workload("teaching_32x4096", decode_steps=steps_budget + 8, seed=seed)
         self.wl = wl
-        S, L, Hq, Hkv, D, B = wl.num_seqs, wl.layers, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+        S, L, Hq, Hkv, D, B = wl.num_seqs, layers, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
         self.S, self.L, self.Hq, self.Hkv, self.D, self.B = S, L, Hq, Hkv, D, B
         N = wl.pool_blocks
         self.N = N
@@ -416,7 +419,7 @@ def main():
     rank, world, dist = dist_init(args.gpus)
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     budget = 2 * (args.warmup + args.steps) + 4
-    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world)
+    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world, args.layers)
     stream = ds.stream
     for _ in range(args.warmup):
         ds.step()
@@ -472,7 +475,8 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "teaching_32x4096", "layers": ds.L, "num_seqs": ds.S, "history": 4096,
+            "config": {"workload": "teaching_32x4096" if ds.L == 32 else f"teaching_32x4096 ({ds.L} layers)",
+                       "layers": ds.L, "num_seqs": ds.S, "history": 4096,
                        "H_q": ds.Hq, "H_kv": ds.Hkv, "head_dim": ds.D, "block_size": ds.B,
                        "pool_blocks_per_layer": ds.N, "kv_pool_gib": round(2 * ds.L * ds.N * ds.B * ds.Hkv * ds.D * 2 / 2**30, 2),
                        "l2": "inputs larger than L2 (KV pool far above 126 MB); no flush",
