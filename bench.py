@@ -7,7 +7,9 @@ H_q 32 / H_kv 8 / d 128, bf16 K/V/Q, block size 16, block tables over a
 shuffled pool of 16 GiB + 10 %.  Per step:
   host allocator append (C++; allocate-or-fail) -> block tables mirrored to
   the device (pinned double buffer) -> copy-on-write copies if any -> slot
-  mapping -> decode plan -> for each layer: kv_append + paged decode attention.
+  mapping -> decode plan -> for each layer: one launch that appends the new
+  token's K/V and runs paged decode attention (--unfused: kv_append, then
+  attention).
 
 Reported (one JSON line from rank 0):
   value        algorithmic HBM bytes of the step / device step time (GB/s);
@@ -15,8 +17,9 @@ Reported (one JSON line from rank 0):
                K/V written + block tables and lengths
   e2e          the same metric with q, new K/V from pinned host buffers and
                the outputs read back to the host inside the timed region
-  roofline     paged decode attention (partition + merge kernels) bytes per
-               launch / its CUDA-event duration, against the measured HBM peak
+  roofline     paged decode attention (one partition-kernel launch per layer,
+               the merge of split requests fused in) bytes per launch / its
+               CUDA-event duration, against the measured HBM peak
   cpu_baseline the float64 oracle on the host cores, on a bounded sample
   clocks       nvidia-smi samples taken during the timed region
 
@@ -50,13 +53,15 @@ METRIC = "paged decode-attn achieved HBM GB/s (frac of peak); decode steps/s at 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=1)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
+    p.add_argument("--unfused", action="store_true",
+                   help="append with a separate kv_append launch instead of folding it into attention")
     p.add_argument("--layers", type=int, default=32,
                    help="layers per step (32 for the workload; fewer only for small profiling captures)")
     return p.parse_args()
@@ -130,7 +135,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
         except Exception:
@@ -174,13 +179,14 @@ class DecodeStep:
     """32-layer decode step through the C ABI; all state resident on the device."""
 
     def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1,
-                 layers: int = 32):
+                 layers: int = 32, fused: bool = True):
         import torch
 
         import paged_kv_cache_358_b200 as pkv
         import workloads as W
 
         self.torch, self.pkv = torch, pkv
+        self.fused = fused
         pkv.set_decode_kernel(kernel)
         wl = W.workload("teaching_32x4096", decode_steps=steps_budget + 8, seed=seed)
         self.wl = wl
@@ -245,9 +251,14 @@ class DecodeStep:
         return self.L * (kv + qo + app + meta) + self.L * cow + 8 * self.S
 
     def attn_bytes_per_launch(self, lens: np.ndarray) -> int:
+        """History K/V read once per KV head, q read, out written, table + length; with the
+        append folded in, also the new K/V rows read and written."""
         e = 2
-        return (int(lens.sum()) * self.Hkv * self.D * e * 2 + self.S * self.Hq * self.D * e * 2
-                + 4 * int(sum(-(-int(n) // self.B) for n in lens)) + 4 * self.S)
+        b = (int(lens.sum()) * self.Hkv * self.D * e * 2 + self.S * self.Hq * self.D * e * 2
+             + 4 * int(sum(-(-int(n) // self.B) for n in lens)) + 4 * self.S)
+        if self.fused:
+            b += self.S * self.Hkv * self.D * e * 2 * 2 + 8 * self.S
+        return b
 
     def step(self, e2e: bool = False):
         torch, pkv = self.torch, self.pkv
@@ -282,17 +293,24 @@ class DecodeStep:
                 self.k_new[i].copy_(self.kn_h[i], non_blocking=True)
                 self.v_new[i].copy_(self.vn_h[i], non_blocking=True)
         for i in range(self.L):
-            pkv.kv_append(self.k_new[i], self.v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
+            if not self.fused:
+                pkv.kv_append(self.k_new[i], self.v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
+                self.launches += 1
             if self.record_attn:
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(self.stream)
-            pkv.paged_decode_attn_run(self.q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
-                                      self.wl.scale, self.out[i], self.ws)
+            if self.fused:
+                pkv.paged_decode_attn_append_run(self.q[i], self.k_new[i], self.v_new[i], self.slots,
+                                                 self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
+                                                 self.wl.scale, self.out[i], self.ws)
+            else:
+                pkv.paged_decode_attn_run(self.q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
+                                          self.wl.scale, self.out[i], self.ws)
             if self.record_attn:
                 e1.record(self.stream)
                 self.attn_events.append((e0, e1))
                 self.attn_bytes.append(self.attn_bytes_per_launch(lens))
-            self.launches += 3
+            self.launches += 1
         if e2e:
             for i in range(self.L):
                 self.out_h[i].copy_(self.out[i], non_blocking=True)
@@ -419,7 +437,7 @@ def main():
     rank, world, dist = dist_init(args.gpus)
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     budget = 2 * (args.warmup + args.steps) + 4
-    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world, args.layers)
+    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world, args.layers, not args.unfused)
     stream = ds.stream
     for _ in range(args.warmup):
         ds.step()
@@ -487,7 +505,8 @@ def main():
                     "ms_per_step": ms_e2e_max / args.steps},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "paged_decode_attn (partition + merge), 32x4096 one layer",
+                         "kernel": ("paged_decode_attn_append_run (append and merge folded in)" if ds.fused else
+                                    "paged_decode_attn_run (merge folded in)") + ", 32x4096, one layer per launch",
                          "avg_launch_us": avg_attn_ms * 1000,
                          "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu,

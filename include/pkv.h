@@ -32,10 +32,11 @@
  * - Block tables: int32 [num_seqs][max_blocks_per_seq], row s holds the
  *   physical ids of request s in logical order; entries past
  *   ceil(seq_lens[s] / B) are never read.
- * - Supported shapes: head_dim * sizeof(dtype) in {128, 256, 512} bytes
- *   (bf16: d = 64, 128, 256; f32: d = 32, 64, 128); block_size in
- *   {1, 2, 4, 8, 16, 32, 64, 128, 256}; num_q_heads % num_kv_heads == 0 with
- *   group G = num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
+ * - Supported decode shapes: bf16 head_dim 64, 128 or 256; f32 head_dim 64
+ *   or 128; block_size 4, 8, 16, 32, 64, 128 or 256; num_q_heads a multiple
+ *   of num_kv_heads (< 4096) with group G = num_q_heads / num_kv_heads in
+ *   {1, 2, 4, 8, 16}.  kv_append and block_copy take any power-of-two block
+ *   size and any row of a multiple of 16 bytes.
  */
 #ifndef PKV_H_
 #define PKV_H_
@@ -82,11 +83,13 @@ const char* pkv_last_cuda_error(void);
  * attention over the contiguous history up to floating-point rounding: the
  * kernels accumulate in fp32 (products of bf16 inputs are exact in fp32).
  *
- * How: a persistent split-sequence partition over all (request, KV head,
- * 16-token tile) units, balanced across every warp of the GPU; each warp keeps
- * an online-softmax state (m, l, o) for the grouped query heads of one KV
- * head, reading each K/V tile once per group through a TMA-fed shared-memory
- * ring; a merge step combines the partial states of requests that were split
+ * How: one persistent kernel launch.  All (request, KV-head group, 16-token
+ * tile) units are split into equal contiguous ranges, one per CTA; the warps
+ * of a CTA take the KV heads of the group over the same tiles, each keeping
+ * an online-softmax state (m, l, o) for the grouped query heads of its KV
+ * head and reading each K/V tile once per group through a TMA-fed
+ * shared-memory ring.  A request split across CTAs is finished by the last
+ * CTA to reach it, which merges the partial states
  * ([P2] exercise "逻辑顺序没错，为什么 attention 输出还是错？": the states merge,
  * per-block outputs do not).
  *
@@ -138,6 +141,31 @@ int pkv_paged_decode_attn_run(const void* q, const void* k_pool, const void* v_p
                               int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
                               int32_t out_dtype, void* workspace, size_t workspace_bytes,
                               pkv_stream_t stream);
+
+/* pkv_kv_append folded into pkv_paged_decode_attn_run: one launch writes each
+ * request's new token into the pools and attends over the history including
+ * it ([P2] section "写满一块，再拿下一块" for the write, section
+ * "分页以后，attention 仍然按完整历史归一化" for the attention).
+ *   k_new, v_new  [num_seqs][num_kv_heads][head_dim], kv_dtype: row s is the
+ *                 new token of request s, which must be the LAST token of its
+ *                 history (position seq_lens[s] - 1, already counted)
+ *   slot_mapping  int64 [num_seqs]: the pool slot of that position (as
+ *                 pkv_slot_mapping gives it); < 0 means request s has no new
+ *                 token in this call; >= num_blocks * block_size is flagged
+ *                 (PKV_ERR_BAD_TABLE) and not written
+ * The result equals pkv_kv_append(k_new, v_new, slot_mapping, num_seqs, ...)
+ * followed by pkv_paged_decode_attn_run(...): the warp that owns a request's
+ * last tile writes the new K/V row to the pool and over the tile row it just
+ * loaded.  Needs a plan in the workspace (pkv_decode_plan);
+ * num_blocks * block_size must be below 2^31. */
+int pkv_paged_decode_attn_append_run(const void* q, const void* k_new, const void* v_new,
+                                     const int64_t* slot_mapping, void* k_pool, void* v_pool,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                     int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                                     int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream);
 
 /* Allocation-free variant of pkv_paged_decode_attn (the pages have no
  * counterpart: this is a deployment convenience).  For callers that cannot

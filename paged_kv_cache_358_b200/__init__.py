@@ -18,7 +18,7 @@ __all__ = [
     "lib", "library_path", "Status", "PkvError",
     "BF16", "F32",
     "decode_workspace_bytes", "paged_decode_attn", "decode_plan", "paged_decode_attn_run",
-    "decode_status", "set_decode_kernel",
+    "decode_status", "set_decode_kernel", "paged_decode_attn_append_run",
     "kv_append", "block_copy", "slot_mapping",
     "BlockAllocator",
 ]
@@ -74,6 +74,9 @@ _SIGS = {
     "pkv_paged_decode_attn_run": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                  _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "pkv_decode_status": (ctypes.c_int, [_vp, _vp]),
+    "pkv_paged_decode_attn_append_run": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32,
+                                                        _i32, _i32, _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz,
+                                                        _vp]),
     "pkv_paged_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                      _i32, _i32, _f32, _i32, _vp, _i32, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
@@ -212,6 +215,27 @@ def paged_decode_attn_run(q, k_pool, v_pool, block_tables, seq_lens, scale: floa
         _dtype_code(k_pool), _dev(out, "out"), _dtype_code(out), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "paged_decode_attn_run")
+    return out
+
+
+def paged_decode_attn_append_run(q, k_new, v_new, slot_mapping, k_pool, v_pool, block_tables, seq_lens,
+                                 scale: float, out, workspace, stream=None):
+    """kv_append(k_new, v_new, slot_mapping) and paged_decode_attn_run in one launch (plan first)."""
+    torch = _torch()
+    S, Hq, Hkv, D, B, N = _attn_args(q, k_pool, v_pool, block_tables, seq_lens, out)
+    if tuple(k_new.shape) != (S, Hkv, D) or tuple(v_new.shape) != (S, Hkv, D):
+        raise ValueError("k_new/v_new must be [num_seqs, num_kv_heads, head_dim]")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape[0] < S:
+        raise TypeError("slot_mapping must be int64 [num_seqs]")
+    if k_new.dtype != k_pool.dtype or v_new.dtype != k_pool.dtype:
+        raise TypeError("dtype mismatch")
+    rc = lib().pkv_paged_decode_attn_append_run(
+        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(slot_mapping, "slot_mapping"),
+        _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), _dev(block_tables, "block_tables"), block_tables.shape[1],
+        _dev(seq_lens, "seq_lens"), S, Hq, Hkv, D, B, N, float(scale), _dtype_code(k_pool), _dev(out, "out"),
+        _dtype_code(out), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc, "paged_decode_attn_append_run")
     return out
 
 

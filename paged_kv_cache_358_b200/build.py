@@ -21,7 +21,8 @@ LIB = os.path.join(HERE, "libpkv.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
               "-Xptxas", "-warn-spills"] + ARCH
-SOURCES = ["pkv_decode.cu", "pkv_kvops.cu", "pkv_alloc.cpp", "pkv_api.cpp"]
+SOURCES = ["pkv_decode.cu", "pkv_decode_bf16_64.cu", "pkv_decode_bf16_128.cu", "pkv_decode_bf16_256.cu",
+           "pkv_decode_f32_64.cu", "pkv_decode_f32_128.cu", "pkv_kvops.cu", "pkv_alloc.cpp", "pkv_api.cpp"]
 
 
 def nvcc() -> str:

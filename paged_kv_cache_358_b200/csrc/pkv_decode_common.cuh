@@ -1,6 +1,5 @@
-// Shared pieces of the decode-attention kernels: workspace layout, the
-// per-warp stream-K worker (its TMA ring, block-table lookahead and pair
-// bookkeeping) and the tile-core interface the FMA and MMA cores implement.
+// Shared pieces of the decode-attention kernels: workspace layout, the work
+// decomposition and the tile-core interface the FMA and MMA cores implement.
 //
 // The method is PagedAttention decode as "PagedAttention：让 KV cache 按需生长"
 // (hs-black.github.io) states it in section
@@ -13,16 +12,19 @@
 // log2 domain (q is pre-multiplied by scale * log2(e)), so every e^x becomes
 // 2^x on the same exponent: the same function, one multiply fewer per score.
 //
-// Work decomposition (our design, not the pages'): a "pair" is (request s,
-// KV head g); a pair's history is cut into 16-token tiles.  All tiles of all
-// pairs form one flattened sequence ordered (s, g, tile), which is split into
-// equal contiguous ranges, one per warp of a persistent grid (a warp-level
-// stream-K).  Each warp walks its range with a private ring of shared-memory
-// stages fed by TMA (cp.async.bulk.tensor), so a long request is spread over
-// many warps and short ones pack together; every warp gets the same number of
-// tiles (+-1) whatever the length mix.  A warp keeps one (m, l, o) state per
-// grouped query head; when its range covers a whole pair it writes the final
-// output, otherwise it writes a partial state that the merge kernel combines.
+// Work decomposition (our design, not the pages'): the KV heads are cut into
+// head groups of HG heads (HG = warps of one CTA); a "pair" is (request s,
+// head group hg) and its history is cut into 16-token tiles.  All tiles of all
+// pairs form one flattened sequence ordered (s, hg, tile), split into equal
+// contiguous ranges, one per CTA of a persistent grid (a stream-K over CTAs).
+// Warp w of a CTA takes KV head hg*HG + w of every tile in the CTA's range, so
+// the warps of a CTA read the same 16 slots of a physical block together: with
+// the [block][slot][head][dim] layout that is one contiguous stretch of HBM
+// per step instead of HG scattered 256-byte rows.  Each warp runs its own ring
+// of shared-memory stages fed by TMA and keeps one (m, l, o) state per grouped
+// query head; when the CTA's range covers a whole pair the warp writes the
+// final output, otherwise a partial state, and the last CTA to finish a split
+// pair merges its partial states (per KV head).
 #pragma once
 
 #include "pkv_device.cuh"
@@ -31,7 +33,7 @@ namespace pkv {
 
 constexpr int kTile = 16;          // tokens per tile
 constexpr int kMaxBoxes = 4;       // TMA boxes per tile (block_size >= 4)
-constexpr int kBatch = 32;         // tiles of table lookahead per warp
+constexpr int kBatch = 16;         // tiles of block-table lookahead per warp
 
 struct WsHeader {
   uint32_t status;
@@ -40,27 +42,34 @@ struct WsHeader {
   int32_t num_kv_heads;
   int32_t head_dim;
   int32_t kv_dtype;
-  int32_t num_workers;
+  int32_t num_workers;     // CTAs of the partition grid
+  int32_t head_groups;     // KV-head groups per request
   int32_t planned;
-  long long total_tiles;
+  int32_t pad;
+  long long total_tiles;   // flattened (request, head group, tile) units
 };
+
+// Partial state of one (CTA, pair, head-in-group): o[G][D], m[G], l[G],
+// padded so every slot starts on a 16-byte boundary.
+constexpr int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
 
 // Workspace layout (byte offsets, each 256-aligned):
 //   header | prefix int32[S+1] (tiles per request, cumulative) |
 //   worker plan int4[NW] {tile_begin, tile_end, s, offset in s} |
-//   partial states float[NW + S*H_kv][part_stride(G, D)]  (o[G][D], m[G], l[G],
-//   padded so every slot starts on a 16-byte boundary)
-constexpr int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
-
+//   arrival counters int32[S*H_kv] (CTAs done with a split (request, KV head)) |
+//   partial states float[(NW + S*NHG) * HG][part_stride(G, D)]
 struct WsLayout {
-  size_t prefix = 0, wplan = 0, partials = 0, total = 0;
+  size_t prefix = 0, wplan = 0, counters = 0, partials = 0, total = 0;
   WsLayout() = default;
   static size_t up(size_t x) { return (x + 255) & ~size_t(255); }
-  WsLayout(int S, int H_kv, int G, int D, int NW) {
+  WsLayout(int S, int H_kv, int HG, int G, int D, int NW) {
+    const int NHG = H_kv / HG;
     prefix = up(sizeof(WsHeader));
     wplan = prefix + up(sizeof(int32_t) * (size_t(S) + 1));
-    partials = wplan + up(sizeof(int4) * size_t(NW));
-    total = partials + up(sizeof(float) * (size_t(NW) + size_t(S) * H_kv) * part_stride(G, D));
+    counters = wplan + up(sizeof(int4) * size_t(NW));
+    partials = counters + up(sizeof(int32_t) * size_t(S) * H_kv);
+    total = partials +
+            up(sizeof(float) * (size_t(NW) + size_t(S) * NHG) * size_t(HG) * part_stride(G, D));
   }
 };
 
@@ -70,13 +79,22 @@ struct DecodeArgs {
   const int32_t* seq_lens;
   void* out;
   char* ws;
-  size_t off_prefix, off_wplan, off_partials;
+  size_t off_prefix, off_wplan, off_counters, off_partials;
   int32_t max_blocks;   // table row stride
   int32_t num_seqs, num_q_heads, num_kv_heads;
+  int32_t head_groups;  // NHG = num_kv_heads / HG
   int32_t block_size, num_blocks;
   int32_t out_dtype;
   int32_t num_workers;
   float scale_log2;     // scale * log2(e)
+  // Folded append (all null when the new tokens were appended separately):
+  // row s of k_new / v_new is request s's new token, the last of its history,
+  // written to pool slot new_slots[s] (< 0: no new token for s).
+  const void* k_new;
+  const void* v_new;
+  const int64_t* new_slots;
+  void* k_pool;
+  void* v_pool;
 };
 
 PKV_DEVINL void store1(void* out, int out_dtype, size_t off, float v) {
@@ -98,11 +116,15 @@ PKV_DEVINL long long range_begin(int v, long long T, int NW) {
 }
 
 // Per-stage metadata written by the issuing lane, read by the consuming warp.
-struct StageMeta {
+struct alignas(16) StageMeta {
   int32_t s;       // request
-  int32_t g;       // KV head
+  int32_t hg;      // head group
   int32_t j;       // tile index within the pair
-  int32_t flags;   // bit 0: first tile of a pair in this warp (q staged); bits 8..: nvalid
+  int32_t flags;   // bit 0: first tile of a pair in this warp (q staged); bit 1: the pair's last
+                   // tile; bits 8..: valid tokens in the tile
+  int32_t nt;      // tiles of the pair
+  int32_t new_slot;  // folded append: pool slot of the pair's new token (< 0: none)
+  int32_t pad[2];
 };
 
 }  // namespace pkv

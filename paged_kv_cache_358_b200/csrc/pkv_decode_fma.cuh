@@ -77,6 +77,9 @@ struct FmaCore {
     }
   }
 
+  // Byte offset of 16-byte unit `unit` of token row t in a K or V tile.
+  static PKV_DEVINL uint32_t row_unit(int t, int unit) { return static_cast<uint32_t>(t * ROWB + unit * 16); }
+
   static PKV_DEVINL void begin_pair(State& st, const char* qsm, float scale_log2, int lane) {
     const int u = lane & (U - 1);
 #pragma unroll

@@ -1,0 +1,527 @@
+// Partition-kernel templates of the decode attention and the host-side
+// launch helpers that instantiate them.  Included by one translation unit per
+// (storage type, head_dim) so the variants compile in parallel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/pkv.h"
+#include <type_traits>
+
+#include "pkv_decode_mma.cuh"
+#include "pkv_host.h"
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// Merge of a split (request, KV head), run by one warp of the last CTA to
+// finish it: combine the partial states (m_u, l_u, o_u) of CTAs u = v0..v1 with
+//   M = max_u m_u,  l = sum_u 2^(m_u - M) l_u,  o = sum_u 2^(m_u - M) o_u,
+// and write o / l -- the online-softmax rescaling rule applied to states.
+// Lanes read the (CTA, head) states of a pass together, so the merge costs a
+// couple of memory round trips, not one per CTA.
+// ---------------------------------------------------------------------------
+// Kept out of line: its load batches need many registers for a moment, and
+// inlined they would raise the register count of the whole streaming loop.
+template <int D, int G, int HG>
+__device__ __noinline__ void merge_pair(const float* partials, long long pp, int w, int v0, int v1, long long T,
+                           int NW, void* out, int out_dtype, size_t out_row, int lane) {
+  constexpr int PS = part_stride(G, D);
+  constexpr int PER = D / 32;   // output elements per lane
+  constexpr int UMAX = 32 / G;  // CTAs per pass: lane i reads (CTA i / G, head i % G)
+  constexpr int NE = UMAX * G;  // (CTA, head) entries per pass (32)
+  constexpr int CH = 16;        // entries whose o slices are loaded per round trip
+  auto slot = [&](int u) { return partials + (static_cast<size_t>(u + pp) * HG + w) * PS; };
+  const int kk = lane % G;
+  float run_m = -INFINITY;  // running max of query head kk (replicated over lanes with equal kk)
+  float run_l = 0.f;        // running sum of query head kk
+  float acc[G][PER];
+#pragma unroll
+  for (int k = 0; k < G; ++k)
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[k][i] = 0.f;
+  for (int u0 = v0; u0 <= v1; u0 += UMAX) {
+    // Every load reads a written slot: CTAs past v1 or without tiles are
+    // replaced by v0 (which always holds a state) and weighted 0, so no load
+    // waits behind a data-dependent branch.  The m/l loads and the first
+    // chunk of o loads go out together.
+    const int uu = u0 + lane / G;
+    const bool valid = uu <= v1 && (T >= NW || range_begin(uu, T, NW) < range_begin(uu + 1, T, NW));
+    const int my_slot = valid ? uu : v0;  // entry `lane` of this pass
+    const float* su = slot(my_slot);
+    float mv = __ldcg(su + G * D + kk);
+    const float lv = __ldcg(su + G * D + G + kk);
+    float vals[CH][PER];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const float* src = slot(__shfl_sync(0xffffffffu, my_slot, c)) + (c % G) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) vals[c][i] = __ldcg(src + i);
+    }
+    if (!valid) mv = -INFINITY;
+    float mk = mv;
+#pragma unroll
+    for (int msk = G; msk < 32; msk <<= 1) mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, msk));
+    const float nm = fmaxf(run_m, mk);
+    const float old_scale = exp2f(run_m - nm);  // 0 on the first pass
+    const float wgt = valid ? exp2f(mv - nm) : 0.f;
+    float wl = wgt * lv;
+#pragma unroll
+    for (int msk = G; msk < 32; msk <<= 1) wl += __shfl_xor_sync(0xffffffffu, wl, msk);
+    run_l = run_l * old_scale + wl;
+    run_m = nm;
+#pragma unroll
+    for (int k = 0; k < G; ++k) {
+      const float sk = __shfl_sync(0xffffffffu, old_scale, k);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[k][i] *= sk;
+    }
+#pragma unroll
+    for (int j0 = 0; j0 < NE; j0 += CH) {
+      if (j0 > 0) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int j = j0 + c;
+          const float* src = slot(__shfl_sync(0xffffffffu, my_slot, j)) + (j % G) * D + lane * PER;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) vals[c][i] = __ldcg(src + i);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int j = j0 + c;
+        const float wj = __shfl_sync(0xffffffffu, wgt, j);  // 0 for replaced entries
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[j % G][i] = fmaf(wj, vals[c][i], acc[j % G][i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const float inv = 1.f / __shfl_sync(0xffffffffu, run_l, k);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) store1(out, out_dtype, out_row + k * D + lane * PER + i, acc[k][i] * inv);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Partition: persistent grid, one stream-K worker per CTA, one KV head per warp.
+// ---------------------------------------------------------------------------
+// One lookahead entry: s, hg | nt << 12, j, flags, new_slot, phys[kMaxBoxes].
+constexpr int kEntryInts = 5 + kMaxBoxes;
+
+template <class Core, int W, int DEPTH>
+struct Smem {
+  static constexpr int kStages = DEPTH * Core::kStageBytes;
+  static constexpr int kScratch = Core::kScratchBytes;
+  static constexpr int kMeta = DEPTH * int(sizeof(StageMeta));
+  static constexpr int kBatchInts = kBatch * kEntryInts;
+  static constexpr int kBatchB = kBatchInts * 4;
+  static constexpr int kBars = DEPTH * 8;
+  static constexpr int kPerWarp =
+      round_up(kStages + kScratch + kMeta + kBatchB + kBars, Core::kAlign);
+  static constexpr int kTotal = W * kPerWarp + Core::kAlign;  // + slack to align the base
+};
+
+constexpr int kSmemPerSM = 232448;  // dynamic shared memory of one SM available to CTAs
+
+// Deepest ring (2..6 stages per warp) whose CTAs fit CPS to an SM.
+template <class Core, int W, int CPS>
+constexpr int pick_depth() {
+  constexpr int lim = kSmemPerSM / CPS - (CPS > 1 ? 1024 : 0);
+  return Smem<Core, W, 6>::kTotal <= lim   ? 6
+         : Smem<Core, W, 5>::kTotal <= lim ? 5
+         : Smem<Core, W, 4>::kTotal <= lim ? 4
+         : Smem<Core, W, 3>::kTotal <= lim ? 3
+                                           : 2;
+}
+
+struct TmaMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+
+template <class Core, int G, int W, int CPS, int DEPTH>
+__global__ void __launch_bounds__(W * 32, CPS)
+    partition_kernel(const __grid_constant__ TmaMaps maps, const DecodeArgs a, int check_S,
+                     int check_Hq, int check_Hkv, int check_D, int check_dtype) {
+  using SM = Smem<Core, W, DEPTH>;
+  constexpr int D = Core::ROWB / Core::ESZ;
+  constexpr int PS = part_stride(G, D);
+  extern __shared__ char smem_raw[];
+  char* base = reinterpret_cast<char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + Core::kAlign - 1) & ~uintptr_t(Core::kAlign - 1));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  char* wbase = base + warp * SM::kPerWarp;
+  char* stages = wbase;
+  float* scratch = reinterpret_cast<float*>(wbase + SM::kStages);
+  StageMeta* meta = reinterpret_cast<StageMeta*>(wbase + SM::kStages + SM::kScratch);
+  int32_t* bt = reinterpret_cast<int32_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta + SM::kBatchB);
+
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
+  uint32_t* status = &hdr->status;
+  if (hdr->planned != 1 || hdr->num_seqs != check_S || hdr->num_q_heads != check_Hq ||
+      hdr->num_kv_heads != check_Hkv || hdr->head_dim != check_D || hdr->kv_dtype != check_dtype ||
+      hdr->num_workers != a.num_workers || hdr->head_groups != a.head_groups) {
+    if (threadIdx.x == 0) record_status(status, kStatusPlanMismatch);
+    return;
+  }
+  const long long T = hdr->total_tiles;
+  const int NW = a.num_workers;
+  const int v = blockIdx.x;  // this CTA's worker id; warp = head within the group
+  const int4 wp = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[v];
+  const int ntiles = wp.y - wp.x;
+
+  const int S = a.num_seqs, Hkv = a.num_kv_heads, NHG = a.head_groups, Bsz = a.block_size;
+  const int Hq = a.num_q_heads;
+  const int box_rows = Bsz < kTile ? Bsz : kTile;
+  const int nbox = kTile / box_rows;  // boxes per tile per chunk
+  const uint64_t pol = policy_evict_first();
+  float* partials = reinterpret_cast<float*>(a.ws + a.off_partials);
+  int32_t* counters = reinterpret_cast<int32_t*>(a.ws + a.off_counters);
+
+  if (ntiles > 0 && lane == 0) {
+    for (int i = 0; i < DEPTH; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // Block-table lookahead, one batch ahead: walk() finds (s, hg, j) of the
+  // next kBatch tiles (lane l takes tile kb + l) and starts their table loads
+  // into registers; commit() stores them to shared memory one batch later,
+  // when the loads have long landed.  The cursor (request cs, offset coff in
+  // its NHG * nt tiles, its length clen) is warp-uniform; seq_lens is only
+  // read when the walk crosses into a new request.
+  int cs = wp.z, coff = wp.w;
+  int clen = ntiles > 0 ? a.seq_lens[cs] : 0;
+  int n_s = 0, n_hg = 0, n_j = 0, n_flags = 0, n_nt = 0;
+  long long n_slot = -1;
+  int n_phys[kMaxBoxes];
+  uint32_t n_have = 0, n_over = 0;  // bit b: box b is read / box b lies past the table row
+  bool n_valid = false;
+
+  auto walk = [&](int kb) {
+    n_valid = lane < kBatch && kb + lane < ntiles;
+    n_have = 0;
+    n_over = 0;
+    if (n_valid) {
+      int s = cs, off = coff + lane, len = clen;
+      int nt = ntiles_of(len);
+      while (off >= NHG * nt) {
+        off -= NHG * nt;
+        if (s + 1 >= S) {  // inconsistent with the plan: stop here
+          record_status(status, kStatusPlanMismatch);
+          off = 0;
+          break;
+        }
+        ++s;
+        len = a.seq_lens[s];
+        nt = ntiles_of(len);
+      }
+      const int hg = nt > 0 ? off / nt : 0;
+      const int j = nt > 0 ? off % nt : 0;
+      const int nblk = (len + Bsz - 1) / Bsz;
+      const int lb0 = (j * kTile) / Bsz;
+      n_s = s;
+      n_hg = hg;
+      n_j = j;
+      n_nt = nt;
+      n_flags = (min(kTile, len - j * kTile) << 8) | (j == nt - 1 ? 2 : 0);
+      n_slot = (a.new_slots != nullptr && j == nt - 1) ? a.new_slots[s] : -1;
+      const int32_t* row = a.block_tables + static_cast<size_t>(s) * a.max_blocks;
+#pragma unroll
+      for (int b = 0; b < kMaxBoxes; ++b) {
+        n_phys[b] = -1;
+        if (b < nbox && lb0 + b < nblk) {
+          if (lb0 + b >= a.max_blocks) {
+            n_over |= 1u << b;
+          } else {
+            n_phys[b] = row[lb0 + b];
+            n_have |= 1u << b;
+          }
+        }
+      }
+      cs = s;
+      coff = off + 1;
+      clen = len;
+    }
+    // the cursor for the next batch comes from the batch's last lane
+    cs = __shfl_sync(0xffffffffu, cs, kBatch - 1);
+    coff = __shfl_sync(0xffffffffu, coff, kBatch - 1);
+    clen = __shfl_sync(0xffffffffu, clen, kBatch - 1);
+  };
+
+  auto commit = [&]() {
+    if (n_valid) {
+      int32_t* e = bt + lane * kEntryInts;
+      e[0] = n_s;
+      e[1] = n_hg | (n_nt << 12);
+      e[2] = n_j;
+      e[3] = n_flags;
+      e[4] = -1;
+      if (n_slot >= static_cast<long long>(a.num_blocks) * Bsz)
+        record_status(status, kStatusBadTable);  // new-token slot outside the pool: not written
+      else if (n_slot >= 0)
+        e[4] = static_cast<int>(n_slot);
+#pragma unroll
+      for (int b = 0; b < kMaxBoxes; ++b) {
+        int phys = -1;
+        if (n_over & (1u << b)) {
+          record_status(status, kStatusBadTable);  // length beyond the table row
+        } else if (n_have & (1u << b)) {
+          phys = n_phys[b];
+          if (phys < 0 || phys >= a.num_blocks) {
+            record_status(status, kStatusBadTable);
+            phys = a.num_blocks;  // out of the tensor map: TMA fills zeros
+          }
+        }
+        e[5 + b] = phys;
+      }
+    }
+    __syncwarp();
+  };
+
+  int last_s = -1, last_hg = -1;
+  auto issue = [&](int k) {
+    if ((k % kBatch) == 0) {
+      commit();               // batch k, loaded during the previous batch
+      walk(k + kBatch);       // start loading batch k + kBatch
+    }
+    if (lane == 0) {
+      const int32_t* e = bt + (k % kBatch) * kEntryInts;
+      const int s = e[0], hg = e[1] & 0xfff, j = e[2];
+      const int head = hg * W + warp;
+      const bool newpair = (s != last_s) || (hg != last_hg);
+      last_s = s;
+      last_hg = hg;
+      const int st = k % DEPTH;
+      char* stage = stages + st * Core::kStageBytes;
+      meta[st].s = s;
+      meta[st].hg = hg;
+      meta[st].j = j;
+      meta[st].flags = e[3] | (newpair ? 1 : 0);
+      meta[st].nt = e[1] >> 12;
+      meta[st].new_slot = e[4];
+      const uint32_t bar = smem_u32(&bars[st]);
+      int nb = 0;
+#pragma unroll
+      for (int b = 0; b < kMaxBoxes; ++b) nb += (b < nbox && e[5 + b] >= 0) ? 1 : 0;
+      const uint32_t box_bytes = static_cast<uint32_t>(box_rows * Core::kChunkRowBytes);
+      uint32_t bytes = 2u * nb * Core::kChunks * box_bytes;
+      if (newpair) bytes += Core::QB;
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bar, bytes);
+      if (newpair) {
+        const char* qsrc = reinterpret_cast<const char*>(a.q) +
+                           (static_cast<size_t>(s) * Hq + static_cast<size_t>(head) * G) * Core::ROWB;
+        bulk_load(smem_u32(stage + Core::kQOff), qsrc, Core::QB, bar);
+      }
+      const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
+#pragma unroll
+      for (int b = 0; b < kMaxBoxes; ++b) {
+        const int phys = e[5 + b];
+        if (b < nbox && phys >= 0) {
+#pragma unroll
+          for (int c = 0; c < Core::kChunks; ++c) {
+            const uint32_t off = c * Core::kChunkBytes + b * box_bytes;
+            tma_load_4d(smem_u32(stage + Core::kKOff + off), &maps.k, c * Core::kBoxInner, slot0, head,
+                        phys, bar, pol);
+            tma_load_4d(smem_u32(stage + Core::kVOff + off), &maps.v, c * Core::kBoxInner, slot0, head,
+                        phys, bar, pol);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  };
+
+  if (ntiles > 0) {
+    walk(0);
+    const int prologue = ntiles < DEPTH ? ntiles : DEPTH;
+    for (int k = 0; k < prologue; ++k) issue(k);
+  }
+
+  // Requests of length 0 produce zeros; CTA v writes those of pairs v, v + NW, ...
+  for (long long p = v; p < static_cast<long long>(S) * NHG; p += NW) {
+    const int s = static_cast<int>(p / NHG), hg = static_cast<int>(p % NHG);
+    if (a.seq_lens[s] != 0) continue;
+    const size_t row = (static_cast<size_t>(s) * Hq + static_cast<size_t>(hg * W + warp) * G) * D;
+    for (int i = lane; i < G * D; i += 32) store1(a.out, a.out_dtype, row + i, 0.f);
+  }
+  if (ntiles <= 0) return;
+
+  typename Core::State state;
+  bool have = false;
+  int ps = 0, phg = 0, jfirst = 0, pnt = 0;
+  long long pstart = 0;
+  bool last_is_end = false;
+
+  auto flush = [&]() {
+    const int head = phg * W + warp;
+    const size_t out_row = (static_cast<size_t>(ps) * Hq + static_cast<size_t>(head) * G) * D;
+    if (jfirst == 0 && last_is_end) {  // the whole pair is in this CTA's range
+      Core::finish(state, true, a.out, a.out_dtype, out_row, nullptr, lane);
+      return;
+    }
+    const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
+    float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
+    Core::finish(state, false, a.out, a.out_dtype, out_row, part, lane);
+    // Count this CTA in for (request, KV head); the last CTA of the pair merges.
+    const size_t ctr = static_cast<size_t>(ps) * Hkv + head;
+    // Release the warp's partial writes and count in (acquire-release at GPU
+    // scope: the last arrival sees every other CTA's partial state).
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[ctr], 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    const int v0 = owner_of(pstart, T, NW), v1 = owner_of(pstart + pnt - 1, T, NW);
+    int expected = v1 - v0 + 1;  // with T >= NW every CTA owns at least one tile
+    if (T < NW) {
+      expected = 0;
+      for (int u = v0; u <= v1; ++u) expected += range_begin(u, T, NW) < range_begin(u + 1, T, NW) ? 1 : 0;
+    }
+    if (prev == expected - 1) {
+      __syncwarp();  // lane 0's acquire orders the whole warp's loads (barrier semantics)
+      merge_pair<D, G, W>(partials, pp, warp, v0, v1, T, NW, a.out, a.out_dtype, out_row, lane);
+      if (lane == 0) atomicExch(&counters[ctr], 0);
+    }
+  };
+
+  for (int k = 0; k < ntiles; ++k) {
+    const int st = k % DEPTH;
+    if (!mbar_wait_bounded(smem_u32(&bars[st]), (k / DEPTH) & 1)) {
+      if (lane == 0) record_status(status, kStatusTimeout);
+      return;
+    }
+    const StageMeta m = meta[st];
+    const char* stage = stages + st * Core::kStageBytes;
+    if (m.flags & 1) {
+      if (have) flush();
+      have = true;
+      ps = m.s;
+      phg = m.hg;
+      jfirst = m.j;
+      pnt = m.nt;
+      pstart = static_cast<long long>(wp.x) + k - m.j;
+      Core::begin_pair(state, stage + Core::kQOff, a.scale_log2, lane);
+    }
+    const int nvalid = m.flags >> 8;
+    last_is_end = (m.flags & 2) != 0;
+    if (m.new_slot >= 0) {
+      // Folded append: this tile holds the pair's new token (row nvalid - 1).
+      // Write its K and V row to the pool and over the stale tile row.
+      const int head = m.hg * W + warp;
+      constexpr int U = Core::ROWB / 16;
+      const size_t src_off = (static_cast<size_t>(m.s) * Hkv + head) * Core::ROWB;
+      const size_t dst_off = (static_cast<size_t>(m.new_slot) * Hkv + head) * Core::ROWB;
+      for (int i = lane; i < 2 * U; i += 32) {
+        const bool is_v = i >= U;
+        const int unit = is_v ? i - U : i;
+        const uint4 val = *reinterpret_cast<const uint4*>(
+            static_cast<const char*>(is_v ? a.v_new : a.k_new) + src_off + unit * 16);
+        *reinterpret_cast<uint4*>(static_cast<char*>(is_v ? a.v_pool : a.k_pool) + dst_off + unit * 16) = val;
+        *reinterpret_cast<uint4*>(const_cast<char*>(stage) + (is_v ? Core::kVOff : Core::kKOff) +
+                                  Core::row_unit(nvalid - 1, unit)) = val;
+      }
+      __syncwarp();
+    }
+    if constexpr (Core::kSwizzle) {
+      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, nvalid, a.scale_log2, lane);
+    } else {
+      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, nvalid, scratch, lane);
+    }
+    __syncwarp();
+    if (k + DEPTH < ntiles) issue(k + DEPTH);
+  }
+  if (have) flush();
+}
+
+
+// ---------------------------------------------------------------------------
+// Host-side launch helpers
+// ---------------------------------------------------------------------------
+struct Geometry {
+  int S, Hq, Hkv, G, D, dtype;
+  int HG, NHG, CPS, NW;
+  WsLayout lay;
+};
+
+extern int g_kernel_choice;  // 0 auto, 1 CUDA-core tiles, 2 tensor-core tiles (bf16)
+
+bool make_pool_map(CUtensorMap* m, const void* pool, int dtype, int D, int B, int Hkv, int N,
+                   int box_inner, int box_rows, bool swizzle);
+
+template <class Core, int G, int W, int CPS>
+int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_pool, const void* v_pool,
+                     cudaStream_t stream) {
+  constexpr int DEPTH = pick_depth<Core, W, CPS>();
+  using SM = Smem<Core, W, DEPTH>;
+  static_assert(SM::kTotal <= kSmemPerSM, "shared memory budget");
+  TmaMaps maps;
+  const int box_rows = args.block_size < kTile ? args.block_size : kTile;
+  if (!make_pool_map(&maps.k, k_pool, geo.dtype, geo.D, args.block_size, geo.Hkv, args.num_blocks,
+                     Core::kBoxInner, box_rows, Core::kSwizzle) ||
+      !make_pool_map(&maps.v, v_pool, geo.dtype, geo.D, args.block_size, geo.Hkv, args.num_blocks,
+                     Core::kBoxInner, box_rows, Core::kSwizzle)) {
+    host::set_error("cuTensorMapEncodeTiled failed");
+    return PKV_ERR_CUDA;
+  }
+  auto kern = partition_kernel<Core, G, W, CPS, DEPTH>;
+  static thread_local int configured_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
+    if (e != cudaSuccess) return host::cuda_fail(e);
+    configured_dev = dev;
+  }
+  kern<<<geo.NW, W * 32, SM::kTotal, stream>>>(maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
+  return host::check_launch();
+}
+
+template <class Core, int G>
+int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, const void* v,
+                cudaStream_t stream) {
+  constexpr int WPS = (Core::ROWB >= 512) ? 4 : 8;
+  switch (geo.HG) {
+    case 8:
+      if constexpr (WPS >= 8) return launch_partition<Core, G, 8, WPS / 8>(geo, args, k, v, stream);
+      break;
+    case 4: return launch_partition<Core, G, 4, WPS / 4>(geo, args, k, v, stream);
+    case 2: return launch_partition<Core, G, 2, WPS / 2>(geo, args, k, v, stream);
+    case 1: return launch_partition<Core, G, 1, WPS>(geo, args, k, v, stream);
+  }
+  return PKV_ERR_INVALID;
+}
+
+// One (storage type, head_dim): dispatch on the group size and the core.
+template <typename T, int D>
+int run_decode(const Geometry& geo, const DecodeArgs& args, const void* k, const void* v,
+               cudaStream_t stream) {
+  auto per_g = [&](auto gc) -> int {
+    constexpr int G = decltype(gc)::value;
+    if constexpr (sizeof(T) == 2 && G <= 8) {
+      if (args.block_size >= 8 && g_kernel_choice != 1)
+        return launch_core<MmaCore<D, G>, G>(geo, args, k, v, stream);
+    }
+    return launch_core<FmaCore<T, D, G>, G>(geo, args, k, v, stream);
+  };
+  switch (geo.G) {
+    case 1: return per_g(std::integral_constant<int, 1>{});
+    case 2: return per_g(std::integral_constant<int, 2>{});
+    case 4: return per_g(std::integral_constant<int, 4>{});
+    case 8: return per_g(std::integral_constant<int, 8>{});
+    case 16: return per_g(std::integral_constant<int, 16>{});
+  }
+  return PKV_ERR_INVALID;
+}
+
+int run_bf16_64(const Geometry&, const DecodeArgs&, const void*, const void*, cudaStream_t);
+int run_bf16_128(const Geometry&, const DecodeArgs&, const void*, const void*, cudaStream_t);
+int run_bf16_256(const Geometry&, const DecodeArgs&, const void*, const void*, cudaStream_t);
+int run_f32_64(const Geometry&, const DecodeArgs&, const void*, const void*, cudaStream_t);
+int run_f32_128(const Geometry&, const DecodeArgs&, const void*, const void*, cudaStream_t);
+
+}  // namespace pkv

@@ -95,6 +95,9 @@ struct MmaCore {
     return static_cast<uint32_t>((unit >> 3) * CHUNKB + t * 128 + (((unit & 7) ^ (t & 7)) << 4));
   }
 
+  // Byte offset of 16-byte unit `unit` of token row t in a K or V tile.
+  static PKV_DEVINL uint32_t row_unit(int t, int unit) { return swz(t, unit); }
+
   static PKV_DEVINL void begin_pair(State& st, const char* qsm, float /*scale_log2*/, int lane) {
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll

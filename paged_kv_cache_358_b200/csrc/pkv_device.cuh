@@ -102,6 +102,13 @@ PKV_DEVINL void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_
       : "memory");
 }
 
+// Atomic add with acquire-release semantics at GPU scope.
+PKV_DEVINL int atomic_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 PKV_DEVINL float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 PKV_DEVINL float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

@@ -358,3 +358,66 @@ def test_empty_batch_and_all_zero_lengths():
     assert torch.count_nonzero(out) == 0
     e = pkv.paged_decode_attn(db.q[:0], db.k_pool, db.v_pool, db.tables[:0], db.seq_lens[:0], wl.scale)
     assert e.shape[0] == 0
+
+
+@pytest.mark.parametrize("B", [4, 16, 64])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_folded_append_equals_append_then_attend(kernel, B, dtype):
+    """pkv_paged_decode_attn_append_run == pkv_kv_append + pkv_paged_decode_attn_run.
+
+    Every other request gets a new token (written at its last position); the
+    rest have slot -1.  Outputs and both pools must match bit for bit, and the
+    output must match the oracle over history + new token."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    from oracle import attention as oatt
+
+    lengths = [1, 5, B, B + 1, 31, 32, 33, 100, 257, 600]
+    Hq, Hkv, D = (8, 2, 64) if dtype == "f32" else (32, 8, 128)
+    wl = W.DecodeWorkload("fold", 1, Hq, Hkv, D, B, dtype, lengths,
+                          pool_blocks=sum(-(-(n + 1) // B) for n in lengths) + 9, seed=40 + B)
+    hb = host_batch(wl)
+    dbs = [device_batch(hb), device_batch(hb)]
+    S = len(lengths)
+    new = [s % 2 == 0 for s in range(S)]
+    g = W.rng(99)
+    kn = W.kv_history(g, wl, S)
+    vn = W.kv_history(g, wl, S)
+    from tests.paged_batch import torch_from_host
+    kn_d, vn_d = torch_from_host(kn), torch_from_host(vn)
+    outs = []
+    for mode, db in zip(("fold", "separate"), dbs):
+        ids = [s for s in range(S) if new[s]]
+        rc, per, copies = db.alloc.append(ids)
+        assert rc == 0 and copies == []
+        mb = max(-(-(n + 1) // B) for n in lengths)
+        tables, lens = db.alloc.fill_tables(list(range(S)), mb)
+        td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+        slots = pkv.slot_mapping(td, torch.from_numpy(lens - 1).cuda(), B)
+        slots[torch.tensor([not x for x in new], device="cuda")] = -1
+        ws = pkv.new_workspace(S, Hq, Hkv, D)
+        pkv.decode_plan(ld, Hq, Hkv, D, pkv.BF16 if dtype == "bf16" else pkv.F32, ws)
+        out = torch.empty((S, Hq, D), dtype=torch.float32, device="cuda")
+        if mode == "fold":
+            pkv.paged_decode_attn_append_run(db.q, kn_d, vn_d, slots, db.k_pool, db.v_pool, td, ld, wl.scale,
+                                             out, ws)
+        else:
+            pkv.kv_append(kn_d, vn_d, slots, db.k_pool, db.v_pool)
+            pkv.paged_decode_attn_run(db.q, db.k_pool, db.v_pool, td, ld, wl.scale, out, ws)
+        assert pkv.decode_status(ws) == 0
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])
+    for a, b in ((dbs[0].k_pool, dbs[1].k_pool), (dbs[0].v_pool, dbs[1].v_pool)):
+        ia = a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32)
+        ib = b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32)
+        assert torch.equal(ia, ib)
+    got = as_f64(outs[0])
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    for s in range(S):
+        kh, vh = hb.k_hist[s], hb.v_hist[s]
+        if new[s]:
+            kh = np.concatenate([kh, kn[s:s + 1]])
+            vh = np.concatenate([vh, vn[s:s + 1]])
+        ref = oatt.dense_decode(hb.q[s], kh, vh, wl.scale)
+        assert np.max(np.abs(got[s] - ref)) <= tol
