@@ -195,6 +195,15 @@ int pkv_paged_decode_attn_noalloc(const void* q, const void* k_pool, const void*
  * PKV_ERR_PLAN_MISMATCH (the first recorded), or PKV_ERR_CUDA. */
 int pkv_decode_status(void* workspace, pkv_stream_t stream);
 
+/* Failure-detection self-test (not a paper operation): launches one warp
+ * that waits on an mbarrier nothing arrives on, through the same bounded wait
+ * the decode kernel uses, for limit_ns nanoseconds (1 .. 1e8); the expiry is
+ * recorded in the workspace status word, so a following pkv_decode_status()
+ * returns PKV_ERR_DEVICE_TIMEOUT.  Nothing faults or hangs: the kernel ends
+ * after the limit and the context stays usable. */
+int pkv_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size_t workspace_bytes,
+                              pkv_stream_t stream);
+
 /* Selects the tile kernel for bf16 storage: 0 = automatic (default),
  * 1 = CUDA-core FMA tiles, 2 = tensor-core (mma.sync bf16) tiles.  fp32
  * storage always uses FMA tiles.  Process-wide; for measurement. */
@@ -237,6 +246,27 @@ int pkv_block_copy(void* const* k_pools, void* const* v_pools, int32_t num_layer
                    int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t dtype,
                    pkv_stream_t stream);
 
+/* pkv_swap_blocks -- preemption by swap ([P2] section
+ * "腾出显存以后，还要付一次恢复成本": release a request's KV and move it over the
+ * host link, then bring it back later, instead of recomputing it).  Moves
+ * blocks[i] of every layer's K and V pool to (to_host = 1) or from
+ * (to_host = 0) a host buffer laid out
+ *     host_buf[n_blocks][num_layers][2 (K, V)][block_size][num_kv_heads][head_dim].
+ *   k_pools,v_pools HOST arrays of num_layers device pool pointers (<= 128)
+ *   blocks          DEVICE int32 [n_blocks]; ids outside [0, num_blocks) are
+ *                   skipped.  Swapping back in may use other block ids (the
+ *                   ones the allocator hands out on re-admission).
+ *   host_buf        page-locked host memory the device can address
+ *                   (cudaHostAlloc, or torch's pinned memory under unified
+ *                   addressing), 16-byte aligned; the kernel reads or writes
+ *                   it directly over the host link.
+ * Asynchronous on `stream`; the host buffer is complete (to_host = 1) or
+ * reusable (to_host = 0) once the stream reaches this point. */
+int pkv_swap_blocks(void* const* k_pools, void* const* v_pools, int32_t num_layers,
+                    const int32_t* blocks, int32_t n_blocks, void* host_buf, int32_t to_host,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                    int32_t dtype, pkv_stream_t stream);
+
 /* pkv_slot_mapping -- slot of each (request row, position) through the block
  * table ([P2] sections "读 token 6，先查表，再找偏移" and
  * "把 token 6 变成真正的内存地址"):
@@ -276,6 +306,7 @@ typedef struct pkv_stats {
   int64_t cow_copies;     /* copy-on-write copies issued                  */
   int64_t alloc_failures; /* requests refused for lack of blocks          */
   int64_t evictions;      /* cached blocks reallocated                    */
+  int64_t prefix_hits;    /* blocks reused by pkv_alloc_add_seq_prefix    */
 } pkv_stats;
 
 /* initial_free_order: host int32 [num_blocks], a permutation of
@@ -346,6 +377,31 @@ int pkv_alloc_check(const pkv_alloc* a);
  * *n_free, *n_cached).  Any pointer may be NULL to skip that part. */
 int pkv_alloc_dump(const pkv_alloc* a, int32_t* refcounts, int32_t* free_order, int32_t* n_free,
                    int32_t* cached_order, int32_t* n_cached);
+
+/* Prefix caching ([P2] sections "请求结束，块就能交给下一位" and
+ * "引用计数管理“谁还在读”，长度管理“哪里能写”": a released full block keeps its
+ * content until it is evicted; section "只读时共用，要写入时再分开": a full-block
+ * hit is shared without a copy; [P3] section 8: the key must name every input
+ * that shaped the state, so the caller computes it (e.g. a hash chained over
+ * the model identity and the block's token ids) and the allocator stores it).
+ *
+ * pkv_alloc_set_block_key: name the content of full block `logical_block` of
+ * live request seq_id with a 64-bit key.  A key names one block and a block
+ * has one key; PKV_ERR_INVALID for a partial block, an unknown request, or a
+ * key/block already bound elsewhere.  Keys are dropped when the block returns
+ * to the free queue or is evicted from the cached set.
+ *
+ * pkv_alloc_add_seq_prefix: admit request seq_id holding n_tokens whose first
+ * n_keys blocks are full blocks with the given keys (n_keys * B <= n_tokens).
+ * Keys are matched in order up to the first miss: a hit on a live block adds
+ * a reference, a hit on a cached block moves it back to active; the remaining
+ * ceil(n_tokens / B) - hits blocks come from the free queue (then the cached
+ * set).  All or nothing: PKV_ERR_NO_BLOCKS leaves everything unchanged.
+ * *n_hit receives the number of reused blocks (their KV need not be
+ * recomputed). */
+int pkv_alloc_set_block_key(pkv_alloc* a, int32_t seq_id, int32_t logical_block, uint64_t key);
+int pkv_alloc_add_seq_prefix(pkv_alloc* a, int32_t seq_id, int32_t n_tokens, const uint64_t* keys,
+                             int32_t n_keys, int32_t* n_hit);
 
 /* Host-side fault injection for failure tests (no device involvement):
  *   PKV_FAULT_ALLOC_FAIL    the next `count` block allocations fail as if

@@ -34,6 +34,19 @@ Readings where the page is silent (each also listed in the design notes):
   to 0 and that holds B valid tokens goes to the cached set (oldest first),
   partial blocks go to the free queue, and allocation evicts the oldest cached
   block only when the free queue is empty.
+
+Prefix caching ([P2] sections "请求结束，块就能交给下一位" and
+"引用计数管理“谁还在读”，长度管理“哪里能写”": released full blocks keep their
+content key until evicted; [P2] section "只读时共用，要写入时再分开": a full-block
+hit is shared without a copy; [P3] section 8: the key must name every input
+that shaped the state -- the caller computes it, the allocator only stores it):
+* ``set_block_key`` gives a full block of a live request a 64-bit content key
+  (a key names one block; a block has one key);
+* ``add_seq_prefix`` admits a request whose leading full blocks carry known
+  keys: matching keys are taken in order until the first miss (a hit on a
+  live block adds a reference, a hit on a cached block moves it back to
+  active), the rest of the blocks come from the free queue; all or nothing;
+* evicting a cached block (allocation with an empty free queue) drops its key.
 """
 from __future__ import annotations
 
@@ -70,7 +83,10 @@ class RefAllocator:
         self.cached = collections.deque()
         self.ref = [0] * num_blocks
         self.seqs: Dict[int, _Seq] = {}
-        self.counters = dict(allocs=0, frees=0, cow_copies=0, alloc_failures=0, evictions=0)
+        self.counters = dict(allocs=0, frees=0, cow_copies=0, alloc_failures=0, evictions=0,
+                             prefix_hits=0)
+        self.key_of = {}      # block -> content key
+        self.block_of = {}    # content key -> block
 
     # -- capacity -----------------------------------------------------------
     def available(self) -> int:
@@ -82,6 +98,9 @@ class RefAllocator:
         else:
             b = self.cached.popleft()
             self.counters["evictions"] += 1
+            k = self.key_of.pop(b, None)
+            if k is not None:
+                del self.block_of[k]
         self.ref[b] = 1
         self.counters["allocs"] += 1
         return b
@@ -162,11 +181,61 @@ class RefAllocator:
             if self.ref[b] == 0:
                 full = i < last or (s.length > 0 and s.length % self.block_size == 0)
                 if self.enable_cache and full:
-                    self.cached.append(b)
+                    self.cached.append(b)      # keeps its content key until evicted
                 else:
                     self.free.append(b)
+                    k = self.key_of.pop(b, None)
+                    if k is not None:
+                        del self.block_of[k]
                 self.counters["frees"] += 1
         return OK
+
+    def set_block_key(self, seq_id: int, logical_block: int, key: int) -> int:
+        """Name the content of a full block of a live request (for later prefix hits)."""
+        if seq_id not in self.seqs:
+            return INVALID
+        s = self.seqs[seq_id]
+        if logical_block < 0 or (logical_block + 1) * self.block_size > s.length:
+            return INVALID                      # only full blocks are shareable
+        b = s.table[logical_block]
+        key = int(key) & 0xFFFFFFFFFFFFFFFF
+        owner = self.block_of.get(key)
+        if owner is not None and owner != b:
+            return INVALID                      # the key already names another block
+        old = self.key_of.get(b)
+        if old is not None and old != key:
+            return INVALID                      # the block already has another key
+        self.key_of[b] = key
+        self.block_of[key] = b
+        return OK
+
+    def add_seq_prefix(self, seq_id: int, n_tokens: int, keys) -> Tuple[int, int]:
+        """Admit a request reusing the cached blocks of its leading full blocks.
+
+        Returns (status, number of leading blocks found in the cache).
+        """
+        keys = [int(k) & 0xFFFFFFFFFFFFFFFF for k in keys]
+        if seq_id in self.seqs or n_tokens < 0 or seq_id < 0 or len(keys) * self.block_size > n_tokens:
+            return INVALID, 0
+        hits = []
+        for k in keys:
+            b = self.block_of.get(k)
+            if b is None:
+                break
+            hits.append(b)
+        need = -(-n_tokens // self.block_size) - len(hits)
+        revived = sum(1 for b in hits if self.ref[b] == 0)
+        if need > self.available() - (revived if self.enable_cache else 0):
+            self.counters["alloc_failures"] += 1
+            return NO_BLOCKS, 0
+        for b in hits:
+            if self.ref[b] == 0:
+                self.cached.remove(b)
+            self.ref[b] += 1
+        self.counters["prefix_hits"] += len(hits)
+        table = hits + [self._take() for _ in range(need)]
+        self.seqs[seq_id] = _Seq(table, n_tokens)
+        return OK, len(hits)
 
     # -- queries ------------------------------------------------------------
     def table(self, seq_id: int) -> List[int]:
@@ -196,4 +265,11 @@ class RefAllocator:
         idle = list(self.free) + list(self.cached)
         if len(set(idle)) != len(idle):
             return False
-        return all(self.ref[b] == 0 for b in idle)
+        if any(self.ref[b] != 0 for b in idle):
+            return False
+        # keys: a bijection between keyed blocks and their keys; free blocks carry none
+        if any(self.block_of.get(k) != b for b, k in self.key_of.items()):
+            return False
+        if len(self.block_of) != len(self.key_of):
+            return False
+        return all(b not in self.key_of for b in self.free)

@@ -19,7 +19,7 @@ __all__ = [
     "BF16", "F32",
     "decode_workspace_bytes", "paged_decode_attn", "decode_plan", "paged_decode_attn_run",
     "decode_status", "set_decode_kernel", "paged_decode_attn_append_run",
-    "kv_append", "block_copy", "slot_mapping",
+    "kv_append", "block_copy", "slot_mapping", "swap_blocks",
     "BlockAllocator",
 ]
 
@@ -55,7 +55,7 @@ class PkvError(RuntimeError):
 class _Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in
                 ("pool", "active", "cached", "free", "seqs", "allocs", "frees", "cow_copies",
-                 "alloc_failures", "evictions")]
+                 "alloc_failures", "evictions", "prefix_hits")]
 
 
 _LIB = None
@@ -80,10 +80,13 @@ _SIGS = {
     "pkv_paged_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                      _i32, _i32, _f32, _i32, _vp, _i32, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
+    "pkv_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_ulonglong, _vp, _sz, _vp]),
     "pkv_kv_append": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_block_copy": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _vp, _i32, _i32, _i32,
                                       _i32, _i32, _i32, _vp]),
     "pkv_slot_mapping": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "pkv_swap_blocks": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _vp, _i32, _vp, _i32, _i32,
+                                       _i32, _i32, _i32, _i32, _vp]),
     "pkv_alloc_create": (_vp, [_i32, _i32, _P32, _i32]),
     "pkv_alloc_destroy": (None, [_vp]),
     "pkv_alloc_add_seq": (ctypes.c_int, [_vp, _i32, _i32]),
@@ -96,6 +99,8 @@ _SIGS = {
     "pkv_alloc_check": (ctypes.c_int, [_vp]),
     "pkv_alloc_dump": (ctypes.c_int, [_vp, _P32, _P32, _P32, _P32, _P32]),
     "pkv_alloc_inject_fault": (ctypes.c_int, [_vp, _i32, _i32]),
+    "pkv_alloc_set_block_key": (ctypes.c_int, [_vp, _i32, _i32, ctypes.c_uint64]),
+    "pkv_alloc_add_seq_prefix": (ctypes.c_int, [_vp, _i32, _i32, ctypes.POINTER(ctypes.c_uint64), _i32, _P32]),
 }
 
 
@@ -286,6 +291,28 @@ def block_copy(k_pools: Sequence, v_pools: Sequence, copies, stream=None) -> Non
     _check(rc, "block_copy")
 
 
+def swap_blocks(k_pools: Sequence, v_pools: Sequence, blocks, host_buf, to_host: bool, stream=None) -> None:
+    """Move blocks (all layers, K and V) to / from a pinned host buffer [n][L][2][B][H_kv][d]."""
+    torch = _torch()
+    L = len(k_pools)
+    if L != len(v_pools) or L == 0:
+        raise ValueError("need the same number (>= 1) of K and V pools")
+    N, B, Hkv, D = k_pools[0].shape
+    if blocks.dtype != torch.int32 or blocks.dim() != 1:
+        raise TypeError("blocks must be int32 [n]")
+    n = blocks.shape[0]
+    if host_buf.is_cuda or not host_buf.is_pinned() or not host_buf.is_contiguous():
+        raise ValueError("host_buf must be contiguous pinned host memory")
+    if host_buf.numel() * host_buf.element_size() < n * L * 2 * B * Hkv * D * k_pools[0].element_size():
+        raise ValueError("host_buf too small")
+    kp = (ctypes.c_void_p * L)(*[_dev(p, "k_pool").value for p in k_pools])
+    vp = (ctypes.c_void_p * L)(*[_dev(p, "v_pool").value for p in v_pools])
+    rc = lib().pkv_swap_blocks(kp, vp, L, _dev(blocks, "blocks") if n else None, n,
+                               ctypes.c_void_p(host_buf.data_ptr()), int(bool(to_host)), Hkv, D, B, N,
+                               _dtype_code(k_pools[0]), _stream(stream))
+    _check(rc, "swap_blocks")
+
+
 def slot_mapping(block_tables, positions, block_size: int, rows=None, out=None, stream=None):
     """slots[i] = table[rows[i]][positions[i] // B] * B + positions[i] % B (int64)."""
     torch = _torch()
@@ -405,6 +432,18 @@ class BlockAllocator:
         nc = np.zeros(1, dtype=np.int32)
         _check(lib().pkv_alloc_dump(self._h, _p32(ref), _p32(fr), _p32(nf), _p32(ca), _p32(nc)), "dump")
         return ref[:self.num_blocks].tolist(), fr[:nf[0]].tolist(), ca[:nc[0]].tolist()
+
+    def set_block_key(self, seq_id: int, logical_block: int, key: int) -> int:
+        return lib().pkv_alloc_set_block_key(self._h, int(seq_id), int(logical_block),
+                                             ctypes.c_uint64(int(key) & 0xFFFFFFFFFFFFFFFF))
+
+    def add_seq_prefix(self, seq_id: int, n_tokens: int, keys: Sequence[int]) -> Tuple[int, int]:
+        k = np.ascontiguousarray(np.asarray([int(x) & 0xFFFFFFFFFFFFFFFF for x in keys], dtype=np.uint64))
+        hit = np.zeros(1, dtype=np.int32)
+        rc = lib().pkv_alloc_add_seq_prefix(self._h, int(seq_id), int(n_tokens),
+                                            k.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64)) if k.size else None,
+                                            int(k.size), _p32(hit))
+        return rc, int(hit[0])
 
     def inject_fault(self, kind: int, count: int = 1) -> None:
         _check(lib().pkv_alloc_inject_fault(self._h, int(kind), int(count)), "inject_fault")

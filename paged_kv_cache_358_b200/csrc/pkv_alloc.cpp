@@ -54,6 +54,37 @@ struct Ring {
   int32_t at(int64_t i) const { return buf[static_cast<size_t>((head + i) % cap())]; }
 };
 
+// Cached set: blocks in release order (oldest first) with O(1) removal of
+// any member, as a prefix hit takes a block from the middle.
+struct LinkedSet {
+  std::vector<int32_t> prev, next;
+  int32_t head = -1, tail = -1;
+  int64_t size = 0;
+  void init(int64_t n) {
+    prev.assign(static_cast<size_t>(n), -1);
+    next.assign(static_cast<size_t>(n), -1);
+  }
+  void push_back(int32_t b) {
+    prev[static_cast<size_t>(b)] = tail;
+    next[static_cast<size_t>(b)] = -1;
+    if (tail >= 0) next[static_cast<size_t>(tail)] = b; else head = b;
+    tail = b;
+    ++size;
+  }
+  void remove(int32_t b) {
+    const int32_t p = prev[static_cast<size_t>(b)], n = next[static_cast<size_t>(b)];
+    if (p >= 0) next[static_cast<size_t>(p)] = n; else head = n;
+    if (n >= 0) prev[static_cast<size_t>(n)] = p; else tail = p;
+    prev[static_cast<size_t>(b)] = next[static_cast<size_t>(b)] = -1;
+    --size;
+  }
+  int32_t pop_front() {
+    const int32_t b = head;
+    remove(b);
+    return b;
+  }
+};
+
 struct Seq {
   std::vector<int32_t> table;
   int32_t length = 0;
@@ -66,8 +97,12 @@ struct pkv_alloc {
   int32_t block_size = 0;
   bool cache = false;
   Ring free_q;
-  Ring cached;
+  LinkedSet cached;
   std::vector<int32_t> ref;
+  std::vector<char> in_cached;       // block is a member of the cached set
+  std::vector<uint64_t> key_of;      // content key of a keyed block
+  std::vector<char> has_key;
+  std::unordered_map<uint64_t, int32_t> block_of;
   std::unordered_map<int32_t, Seq> seqs;
   int64_t active = 0;  // blocks with refcount > 0
   pkv_stats ctr{};
@@ -82,12 +117,21 @@ struct pkv_alloc {
     return available() >= n;
   }
 
+  void drop_key(int32_t b) {
+    if (has_key[static_cast<size_t>(b)]) {
+      block_of.erase(key_of[static_cast<size_t>(b)]);
+      has_key[static_cast<size_t>(b)] = 0;
+    }
+  }
+
   int32_t take() {
     int32_t b;
     if (free_q.size > 0) {
       b = free_q.pop_front();
     } else {
       b = cached.pop_front();
+      in_cached[static_cast<size_t>(b)] = 0;
+      drop_key(b);  // eviction forgets the content
       ++ctr.evictions;
     }
     ref[static_cast<size_t>(b)] = 1;
@@ -115,6 +159,9 @@ pkv_alloc* pkv_alloc_create(int32_t num_blocks, int32_t block_size,
     a->free_q.init(num_blocks);
     a->cached.init(num_blocks);
     a->ref.assign(static_cast<size_t>(num_blocks), 0);
+    a->in_cached.assign(static_cast<size_t>(num_blocks), 0);
+    a->key_of.assign(static_cast<size_t>(num_blocks), 0);
+    a->has_key.assign(static_cast<size_t>(num_blocks), 0);
     if (initial_free_order) {
       std::vector<char> seen(static_cast<size_t>(num_blocks), 0);
       for (int32_t i = 0; i < num_blocks; ++i) {
@@ -252,10 +299,13 @@ int pkv_alloc_free_seq(pkv_alloc* a, int32_t seq_id) {
       --a->active;
       ++a->ctr.frees;
       const bool full = i < last || (s.length > 0 && s.length % B == 0);
-      if (a->cache && full)
-        a->cached.push_back(b);
-      else
+      if (a->cache && full) {
+        a->cached.push_back(b);  // keeps its content key until evicted
+        a->in_cached[static_cast<size_t>(b)] = 1;
+      } else {
         a->free_q.push_back(b);
+        a->drop_key(b);
+      }
     }
   }
   a->seqs.erase(it);
@@ -338,11 +388,25 @@ int pkv_alloc_check(const pkv_alloc* a) {
     if (idle[static_cast<size_t>(b)] || a->ref[static_cast<size_t>(b)] != 0) return PKV_ERR_INVALID;
     idle[static_cast<size_t>(b)] = 1;
   }
-  for (int64_t i = 0; i < a->cached.size; ++i) {
-    const int32_t b = a->cached.at(i);
-    if (idle[static_cast<size_t>(b)] || a->ref[static_cast<size_t>(b)] != 0) return PKV_ERR_INVALID;
+  int64_t n_cached = 0;
+  for (int32_t b = a->cached.head; b >= 0; b = a->cached.next[static_cast<size_t>(b)]) {
+    if (++n_cached > a->num_blocks) return PKV_ERR_INVALID;  // a cycle
+    if (idle[static_cast<size_t>(b)] || a->ref[static_cast<size_t>(b)] != 0 ||
+        !a->in_cached[static_cast<size_t>(b)])
+      return PKV_ERR_INVALID;
     idle[static_cast<size_t>(b)] = 1;
   }
+  if (n_cached != a->cached.size) return PKV_ERR_INVALID;
+  size_t keyed = 0;
+  for (size_t b = 0; b < N; ++b) {
+    if (!a->has_key[b]) continue;
+    ++keyed;
+    auto it = a->block_of.find(a->key_of[b]);
+    if (it == a->block_of.end() || it->second != static_cast<int32_t>(b)) return PKV_ERR_INVALID;
+  }
+  if (keyed != a->block_of.size()) return PKV_ERR_INVALID;
+  for (int64_t i = 0; i < a->free_q.size; ++i)
+    if (a->has_key[static_cast<size_t>(a->free_q.at(i))]) return PKV_ERR_INVALID;
   return PKV_OK;
 }
 
@@ -354,9 +418,79 @@ int pkv_alloc_dump(const pkv_alloc* a, int32_t* refcounts, int32_t* free_order, 
   if (free_order)
     for (int64_t i = 0; i < a->free_q.size; ++i) free_order[i] = a->free_q.at(i);
   if (n_free) *n_free = static_cast<int32_t>(a->free_q.size);
-  if (cached_order)
-    for (int64_t i = 0; i < a->cached.size; ++i) cached_order[i] = a->cached.at(i);
+  if (cached_order) {
+    int64_t i = 0;
+    for (int32_t b = a->cached.head; b >= 0; b = a->cached.next[static_cast<size_t>(b)]) cached_order[i++] = b;
+  }
   if (n_cached) *n_cached = static_cast<int32_t>(a->cached.size);
+  return PKV_OK;
+}
+
+int pkv_alloc_set_block_key(pkv_alloc* a, int32_t seq_id, int32_t logical_block, uint64_t key) {
+  if (!a) return PKV_ERR_INVALID;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PKV_ERR_INVALID;
+  const Seq& s = it->second;
+  if (logical_block < 0 ||
+      (static_cast<int64_t>(logical_block) + 1) * a->block_size > s.length)
+    return PKV_ERR_INVALID;  // only full blocks are shareable
+  const int32_t b = s.table[static_cast<size_t>(logical_block)];
+  auto owner = a->block_of.find(key);
+  if (owner != a->block_of.end() && owner->second != b) return PKV_ERR_INVALID;
+  if (a->has_key[static_cast<size_t>(b)] && a->key_of[static_cast<size_t>(b)] != key) return PKV_ERR_INVALID;
+  try {
+    a->block_of[key] = b;
+  } catch (...) {
+    return PKV_ERR_INVALID;
+  }
+  a->key_of[static_cast<size_t>(b)] = key;
+  a->has_key[static_cast<size_t>(b)] = 1;
+  return PKV_OK;
+}
+
+int pkv_alloc_add_seq_prefix(pkv_alloc* a, int32_t seq_id, int32_t n_tokens, const uint64_t* keys,
+                             int32_t n_keys, int32_t* n_hit) {
+  if (!a || seq_id < 0 || n_tokens < 0 || n_keys < 0 || (n_keys > 0 && !keys)) return PKV_ERR_INVALID;
+  if (a->seqs.count(seq_id)) return PKV_ERR_INVALID;
+  if (static_cast<int64_t>(n_keys) * a->block_size > n_tokens) return PKV_ERR_INVALID;
+  std::vector<int32_t> hits;
+  int64_t revived = 0;
+  for (int32_t i = 0; i < n_keys; ++i) {
+    auto it = a->block_of.find(keys[i]);
+    if (it == a->block_of.end()) break;
+    hits.push_back(it->second);
+    if (a->ref[static_cast<size_t>(it->second)] == 0) ++revived;
+  }
+  const int64_t need = (static_cast<int64_t>(n_tokens) + a->block_size - 1) / a->block_size -
+                       static_cast<int64_t>(hits.size());
+  const int64_t avail = a->available() - (a->cache ? revived : 0);
+  if (need > 0 && (a->fault_alloc_fail > 0 || need > avail)) {
+    a->consume_alloc_fault();
+    ++a->ctr.alloc_failures;
+    if (n_hit) *n_hit = 0;
+    return PKV_ERR_NO_BLOCKS;
+  }
+  try {
+    Seq s;
+    s.table.reserve(hits.size() + static_cast<size_t>(need));
+    for (int32_t b : hits) {
+      int32_t& r = a->ref[static_cast<size_t>(b)];
+      if (r == 0) {  // a cached block comes back to active
+        a->cached.remove(b);
+        a->in_cached[static_cast<size_t>(b)] = 0;
+        ++a->active;
+      }
+      r += 1;
+      s.table.push_back(b);
+    }
+    for (int64_t i = 0; i < need; ++i) s.table.push_back(a->take());
+    s.length = n_tokens;
+    a->seqs.emplace(seq_id, std::move(s));
+  } catch (...) {
+    return PKV_ERR_INVALID;
+  }
+  a->ctr.prefix_hits += static_cast<int64_t>(hits.size());
+  if (n_hit) *n_hit = static_cast<int32_t>(hits.size());
   return PKV_OK;
 }
 

@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
   // request is the last s with NHG * P[s] <= start (skipping empty requests).
   for (int v = tid; v < NW; v += kPlanThreads) {
     if (T == 0) {
-      wplan[v] = make_int4(0, 0, 0, 0);
+      wplan[2 * v] = make_int4(0, 0, 0, 0);
+      wplan[2 * v + 1] = make_int4(0, 0, 0, 0);
       continue;
     }
     const long long a = range_begin(v, T, NW);
@@ -97,8 +98,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
       const int mid = (lo + hi + 1) >> 1;
       if (static_cast<long long>(P[mid]) * NHG <= a) lo = mid; else hi = mid - 1;
     }
-    wplan[v] = make_int4(static_cast<int>(a), static_cast<int>(b), lo,
-                         static_cast<int>(a - static_cast<long long>(P[lo]) * NHG));
+    wplan[2 * v] = make_int4(static_cast<int>(a), static_cast<int>(b), lo,
+                             static_cast<int>(a - static_cast<long long>(P[lo]) * NHG));
+    wplan[2 * v + 1] = make_int4(seq_lens[lo], 0, 0, 0);  // saves the worker a dependent load
   }
   if (tid == 0) {
     hdr->num_seqs = S;
@@ -193,15 +195,14 @@ bool shape_ok(int Hq, int Hkv, int D, int dtype) {
   return false;
 }
 
-// Warps per SM: 8 for rows of up to 256 bytes, 4 for 512-byte rows (their
-// stages are twice as large).  A CTA holds one head group of HG warps; the
-// plan and every kernel variant agree on these numbers.
+// Workers per SM: 8 for rows of up to 256 bytes, 4 for 512-byte rows (their
+// stages are twice as large).  Each worker is a one-warp CTA (head group of
+// one KV head): measured on the 32 x 4096 decode, one-warp workers stream
+// faster than CTAs whose warps share a block's KV heads (102 vs 110 us per
+// layer), so the head-group width is 1.  The plan and every kernel variant
+// agree on these numbers.
 int warps_per_sm(int D, int dtype) { return D * esize(dtype) >= 512 ? 4 : 8; }
-int head_group(int Hkv, int wps) {
-  for (int hg = wps; hg > 1; hg >>= 1)
-    if (Hkv % hg == 0) return hg;
-  return 1;
-}
+int head_group(int /*Hkv*/, int /*wps*/) { return 1; }
 
 bool geometry(int S, int Hq, int Hkv, int D, int dtype, Geometry* g) {
   if (S < 0 || !valid_dtype(dtype) || !shape_ok(Hq, Hkv, D, dtype)) return false;
@@ -396,6 +397,36 @@ int pkv_decode_status(void* workspace, pkv_stream_t stream) {
   if (st & kStatusTimeout) return PKV_ERR_DEVICE_TIMEOUT;
   if (st & kStatusPlanMismatch) return PKV_ERR_PLAN_MISMATCH;
   return PKV_OK;
+}
+
+}  // extern "C"
+
+namespace pkv {
+
+// One warp waits on an mbarrier that nothing arrives on, through the same
+// bounded wait the decode kernel uses, and records the timeout.
+__global__ void bounded_wait_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    pkv::mbar_init(pkv::smem_u32(&bar), 1);
+    pkv::fence_mbar_init();
+  }
+  __syncwarp();
+  if (!pkv::mbar_wait_bounded(pkv::smem_u32(&bar), 0, limit_ns) && threadIdx.x == 0)
+    pkv::record_status(status, pkv::kStatusTimeout);
+}
+
+}  // namespace pkv
+
+extern "C" {
+
+int pkv_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size_t workspace_bytes,
+                              pkv_stream_t stream) {
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < sizeof(WsHeader)) return PKV_ERR_INVALID;
+  if (limit_ns == 0 || limit_ns > 100000000ull) return PKV_ERR_INVALID;  // at most 0.1 s
+  pkv::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      &reinterpret_cast<WsHeader*>(workspace)->status, limit_ns);
+  return host::check_launch();
 }
 
 int pkv_set_decode_kernel(int32_t which) {

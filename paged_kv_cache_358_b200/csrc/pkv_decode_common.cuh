@@ -12,19 +12,18 @@
 // log2 domain (q is pre-multiplied by scale * log2(e)), so every e^x becomes
 // 2^x on the same exponent: the same function, one multiply fewer per score.
 //
-// Work decomposition (our design, not the pages'): the KV heads are cut into
-// head groups of HG heads (HG = warps of one CTA); a "pair" is (request s,
-// head group hg) and its history is cut into 16-token tiles.  All tiles of all
-// pairs form one flattened sequence ordered (s, hg, tile), split into equal
-// contiguous ranges, one per CTA of a persistent grid (a stream-K over CTAs).
-// Warp w of a CTA takes KV head hg*HG + w of every tile in the CTA's range, so
-// the warps of a CTA read the same 16 slots of a physical block together: with
-// the [block][slot][head][dim] layout that is one contiguous stretch of HBM
-// per step instead of HG scattered 256-byte rows.  Each warp runs its own ring
-// of shared-memory stages fed by TMA and keeps one (m, l, o) state per grouped
-// query head; when the CTA's range covers a whole pair the warp writes the
-// final output, otherwise a partial state, and the last CTA to finish a split
-// pair merges its partial states (per KV head).
+// Work decomposition (our design, not the pages'): a "pair" is (request s,
+// KV-head group hg) and its history is cut into 16-token tiles.  All tiles of
+// all pairs form one flattened sequence ordered (s, hg, tile), split into
+// equal contiguous ranges, one per CTA of a persistent grid (a stream-K over
+// CTAs), so every CTA streams the same number of tiles whatever the length
+// mix.  Warp w of a CTA takes KV head hg*HG + w of each tile in the range; the
+// library runs one-warp CTAs (HG = 1, eight per SM), the width that measured
+// fastest.  Each warp runs its own ring of shared-memory stages fed by TMA and
+// keeps one (m, l, o) state per grouped query head; when the CTA's range
+// covers a whole pair the warp writes the final output, otherwise a partial
+// state, and the last CTA to finish a split (request, KV head) merges the
+// partial states.
 #pragma once
 
 #include "pkv_device.cuh"
@@ -33,7 +32,7 @@ namespace pkv {
 
 constexpr int kTile = 16;          // tokens per tile
 constexpr int kMaxBoxes = 4;       // TMA boxes per tile (block_size >= 4)
-constexpr int kBatch = 16;         // tiles of block-table lookahead per warp
+constexpr int kBatch = 32;         // tiles of block-table lookahead per warp
 
 struct WsHeader {
   uint32_t status;
@@ -55,7 +54,7 @@ constexpr int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
 
 // Workspace layout (byte offsets, each 256-aligned):
 //   header | prefix int32[S+1] (tiles per request, cumulative) |
-//   worker plan int4[NW] {tile_begin, tile_end, s, offset in s} |
+//   worker plan int4[2*NW] {tile_begin, tile_end, s, offset in s}, {len(s), 0, 0, 0} |
 //   arrival counters int32[S*H_kv] (CTAs done with a split (request, KV head)) |
 //   partial states float[(NW + S*NHG) * HG][part_stride(G, D)]
 struct WsLayout {
@@ -66,7 +65,7 @@ struct WsLayout {
     const int NHG = H_kv / HG;
     prefix = up(sizeof(WsHeader));
     wplan = prefix + up(sizeof(int32_t) * (size_t(S) + 1));
-    counters = wplan + up(sizeof(int4) * size_t(NW));
+    counters = wplan + up(2 * sizeof(int4) * size_t(NW));
     partials = counters + up(sizeof(int32_t) * size_t(S) * H_kv);
     total = partials +
             up(sizeof(float) * (size_t(NW) + size_t(S) * NHG) * size_t(HG) * part_stride(G, D));

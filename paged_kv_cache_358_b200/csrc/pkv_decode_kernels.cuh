@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(W * 32, CPS)
   const long long T = hdr->total_tiles;
   const int NW = a.num_workers;
   const int v = blockIdx.x;  // this CTA's worker id; warp = head within the group
-  const int4 wp = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[v];
+  const int4 wp = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[2 * v];
+  const int first_len = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[2 * v + 1].x;
   const int ntiles = wp.y - wp.x;
 
   const int S = a.num_seqs, Hkv = a.num_kv_heads, NHG = a.head_groups, Bsz = a.block_size;
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
   // its NHG * nt tiles, its length clen) is warp-uniform; seq_lens is only
   // read when the walk crosses into a new request.
   int cs = wp.z, coff = wp.w;
-  int clen = ntiles > 0 ? a.seq_lens[cs] : 0;
+  int clen = first_len;
   int n_s = 0, n_hg = 0, n_j = 0, n_flags = 0, n_nt = 0;
   long long n_slot = -1;
   int n_phys[kMaxBoxes];
@@ -485,15 +486,8 @@ template <class Core, int G>
 int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, const void* v,
                 cudaStream_t stream) {
   constexpr int WPS = (Core::ROWB >= 512) ? 4 : 8;
-  switch (geo.HG) {
-    case 8:
-      if constexpr (WPS >= 8) return launch_partition<Core, G, 8, WPS / 8>(geo, args, k, v, stream);
-      break;
-    case 4: return launch_partition<Core, G, 4, WPS / 4>(geo, args, k, v, stream);
-    case 2: return launch_partition<Core, G, 2, WPS / 2>(geo, args, k, v, stream);
-    case 1: return launch_partition<Core, G, 1, WPS>(geo, args, k, v, stream);
-  }
-  return PKV_ERR_INVALID;
+  if (geo.HG != 1) return PKV_ERR_INVALID;
+  return launch_partition<Core, G, 1, WPS>(geo, args, k, v, stream);
 }
 
 // One (storage type, head_dim): dispatch on the group size and the core.

@@ -62,15 +62,15 @@ PKV_DEVINL bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier, for at most kWaitLimitNs.  Returns
+// Wait for phase `parity` of an mbarrier, for at most limit_ns.  Returns
 // false (and the caller records kStatusTimeout) if the phase never completed.
-PKV_DEVINL bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+PKV_DEVINL bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0 && globaltimer() - t0 > kWaitLimitNs) return false;
+    if ((++spins & 63u) == 0 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 

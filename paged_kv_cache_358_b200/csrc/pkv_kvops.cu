@@ -11,7 +11,10 @@
 //     of every layer before the write (sections "只读时共用，要写入时再分开" and
 //     "一次写入，为什么会先少掉一个空闲块？"); stream order makes the copy visible
 //     before the append that follows it (section "先确保分配成功，再改变可见状态").
-// All three are pure data movement; each thread moves 16-byte vectors.
+//   * preemption by swap moves a request's blocks (every layer, K and V) to a
+//     pinned host buffer and back, the alternative to recompute weighed in
+//     section "腾出显存以后，还要付一次恢复成本".
+// All four are pure data movement; each thread moves 16-byte vectors.
 #include <cuda_runtime.h>
 
 #include "../../include/pkv.h"
@@ -56,6 +59,24 @@ __global__ void __launch_bounds__(256) block_copy_kernel(const __grid_constant__
   uint4* d = pool + static_cast<long long>(dst) * B * row_vec;
   const int n = nv * row_vec;
   for (int i = threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+// grid (block, layer, tensor): move one block of one layer's K or V between
+// the pool and a host buffer laid out [n][layer][K,V][B * H_kv * d].
+__global__ void __launch_bounds__(256) swap_kernel(const __grid_constant__ PoolPtrs pools,
+                                                   const int32_t* __restrict__ blocks, int num_layers,
+                                                   uint4* __restrict__ host, int block_vec, int N,
+                                                   int to_host) {
+  const int i = blockIdx.x, layer = blockIdx.y, is_v = blockIdx.z;
+  const int b = blocks[i];
+  if (b < 0 || b >= N) return;
+  uint4* pool = (is_v ? pools.v[layer] : pools.k[layer]) + static_cast<long long>(b) * block_vec;
+  uint4* h = host + ((static_cast<long long>(i) * num_layers + layer) * 2 + is_v) * block_vec;
+  if (to_host) {
+    for (int j = threadIdx.x; j < block_vec; j += blockDim.x) h[j] = pool[j];
+  } else {
+    for (int j = threadIdx.x; j < block_vec; j += blockDim.x) pool[j] = h[j];
+  }
 }
 
 __global__ void slot_mapping_kernel(const int32_t* __restrict__ tables, int max_blocks,
@@ -130,6 +151,32 @@ int pkv_block_copy(void* const* k_pools, void* const* v_pools, int32_t num_layer
   dim3 grid(static_cast<unsigned>(n_copies), static_cast<unsigned>(num_layers), 2);
   block_copy_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       p, copies, static_cast<int>(row_bytes / 16), block_size, num_blocks);
+  return host::check_launch();
+}
+
+int pkv_swap_blocks(void* const* k_pools, void* const* v_pools, int32_t num_layers,
+                    const int32_t* blocks, int32_t n_blocks, void* host_buf, int32_t to_host,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                    int32_t dtype, pkv_stream_t stream) {
+  const int es = esize(dtype);
+  if (!es || n_blocks < 0 || num_layers < 1 || num_layers > kMaxLayers || num_kv_heads <= 0 ||
+      head_dim <= 0 || num_blocks < 0 || !pow2_block(block_size) || (to_host != 0 && to_host != 1))
+    return PKV_ERR_INVALID;
+  const long long block_bytes = static_cast<long long>(block_size) * num_kv_heads * head_dim * es;
+  if (block_bytes % 16) return PKV_ERR_INVALID;
+  if (n_blocks == 0) return PKV_OK;
+  if (!k_pools || !v_pools || !blocks || !host_buf || !aligned16(host_buf)) return PKV_ERR_INVALID;
+  PoolPtrs p{};
+  for (int l = 0; l < num_layers; ++l) {
+    if (!k_pools[l] || !v_pools[l] || !aligned16(k_pools[l]) || !aligned16(v_pools[l]))
+      return PKV_ERR_INVALID;
+    p.k[l] = static_cast<uint4*>(k_pools[l]);
+    p.v[l] = static_cast<uint4*>(v_pools[l]);
+  }
+  dim3 grid(static_cast<unsigned>(n_blocks), static_cast<unsigned>(num_layers), 2);
+  swap_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      p, blocks, num_layers, static_cast<uint4*>(host_buf), static_cast<int>(block_bytes / 16), num_blocks,
+      to_host);
   return host::check_launch();
 }
 

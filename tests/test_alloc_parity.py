@@ -172,3 +172,73 @@ def test_fill_tables_and_errors():
         a.fill_tables([7], 4)
     assert a.add_seq(5, 1) == pkv.Status.INVALID and a.add_seq(-1, 1) == pkv.Status.INVALID
     assert a.append([]) == (0, [], [])
+
+
+@pytest.mark.parametrize("seed,cache", [(10, True), (11, False), (12, True)])
+def test_prefix_cache_random_sequences_bit_exact(seed, cache):
+    """Keys on full blocks, prefix admissions (hits on live and cached blocks), evictions."""
+    rnd = random.Random(seed)
+    N, B = 48, 4
+    order = rnd.sample(range(N), N)
+    ref = RefAllocator(N, B, free_order=order, enable_cache=cache)
+    cpp = pkv.BlockAllocator(N, B, free_order=order, enable_cache=cache)
+    live, nxt = [], 0
+    prompts = {}      # seq -> list of block keys of its full blocks (prompt "tokens")
+    for step in range(1500):
+        op = rnd.random()
+        if op < 0.25 or not live:
+            # a prompt built from a few shared prefixes: keys chained like a content hash
+            base = rnd.randint(0, 5)
+            nfull = rnd.randint(0, 4)
+            keys = [(base * 1000 + i) * 7919 for i in range(nfull)]
+            n = nfull * B + rnd.randint(0, B)
+            r1 = ref.add_seq_prefix(nxt, n, keys)
+            r2 = cpp.add_seq_prefix(nxt, n, keys)
+            assert r1 == r2
+            if r1[0] == 0:
+                live.append(nxt)
+                prompts[nxt] = keys
+                for i, k in enumerate(keys):            # publish the keys of its full blocks
+                    a, b = ref.set_block_key(nxt, i, k), cpp.set_block_key(nxt, i, k)
+                    assert a == b
+            nxt += 1
+        elif op < 0.35:
+            sid = rnd.choice(live)
+            lb = rnd.randint(0, 5)
+            key = rnd.randint(0, 2 ** 64 - 1)
+            assert ref.set_block_key(sid, lb, key) == cpp.set_block_key(sid, lb, key)
+        elif op < 0.75:
+            ids = rnd.sample(live, rnd.randint(1, len(live)))
+            assert ref.append(ids) == cpp.append(ids)
+        else:
+            sid = live.pop(rnd.randrange(len(live)))
+            assert ref.free_seq(sid) == cpp.free_seq(sid) == 0
+        _same(ref, cpp, live)
+        assert ref.stats()["prefix_hits"] == cpp.stats()["prefix_hits"]
+
+
+def test_prefix_hit_revives_cached_block_and_eviction_forgets():
+    """A released full block stays cached with its key; a later request with the same
+    prefix reuses it without a copy; once evicted, the key no longer hits."""
+    for A in (RefAllocator, pkv.BlockAllocator):
+        a = A(4, 4, enable_cache=True)
+        assert a.add_seq_prefix(0, 8, [111, 222]) == (0, 0)     # cold: no hits
+        assert a.set_block_key(0, 0, 111) == 0 and a.set_block_key(0, 1, 222) == 0
+        assert a.set_block_key(0, 1, 333) == 2                   # a block has one key
+        t0 = a.table(0)
+        assert a.free_seq(0) == 0
+        st = a.stats()
+        assert (st["active"], st["cached"], st["free"]) == (0, 2, 2)
+        assert a.add_seq_prefix(1, 9, [111, 222]) == (0, 2)     # both blocks reused
+        assert a.table(1)[:2] == t0
+        st = a.stats()
+        assert (st["active"], st["cached"], st["free"], st["prefix_hits"]) == (3, 0, 1, 2)
+        assert a.add_seq_prefix(2, 8, [111, 999]) == (0, 1)     # live hit shares, miss stops
+        assert a.table(2)[0] == t0[0] and a.check()
+        assert a.free_seq(1) == 0 and a.free_seq(2) == 0
+        # fill the pool so the cached blocks get evicted, then the keys miss
+        assert a.add_seq(3, 16) == 0
+        assert a.stats()["evictions"] >= 2
+        assert a.free_seq(3) == 0
+        assert a.add_seq_prefix(4, 4, [111]) == (0, 0)
+        assert a.check()

@@ -421,3 +421,28 @@ def test_folded_append_equals_append_then_attend(kernel, B, dtype):
             vh = np.concatenate([vh, vn[s:s + 1]])
         ref = oatt.dense_decode(hb.q[s], kh, vh, wl.scale)
         assert np.max(np.abs(got[s] - ref)) <= tol
+
+
+def test_bounded_device_wait_reports_timeout():
+    """A wait that nothing satisfies ends after its limit with a status, not a hang."""
+    import time
+
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    t0 = time.perf_counter()
+    rc = pkv.lib().pkv_selftest_bounded_wait(5_000_000, ws.data_ptr(), ws.numel(),
+                                              torch.cuda.current_stream().cuda_stream)
+    assert rc == pkv.Status.OK
+    assert pkv.decode_status(ws) == pkv.Status.DEVICE_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert pkv.decode_status(ws) == pkv.Status.OK        # cleared by the read
+    # the context is still usable: a normal decode runs afterwards
+    wl = W.workload("tiny")
+    hb = host_batch(wl)
+    db = device_batch(hb)
+    got = as_f64(_run(db, hb, torch.float32))
+    from tests.paged_batch import oracle_out
+    assert np.max(np.abs(got - oracle_out(hb))) <= TOL_F32

@@ -163,3 +163,92 @@ def test_append_rejects_bad_arguments():
     rc = L.pkv_kv_append(k.data_ptr() + 2, k.data_ptr(), s.data_ptr(), 1, kp.data_ptr(), kp.data_ptr(), 2,
                          64, 8, 4, 0, None)           # misaligned
     assert rc == pkv.Status.INVALID
+
+
+def test_preempt_by_swap_round_trip():
+    """Preempt a request: swap its blocks (every layer, K and V) to pinned host memory,
+    release them, let another request overwrite the pool, re-admit it (new block ids)
+    and swap back in; the KV bytes and the attention output are unchanged."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    L, N, B, Hkv, D, Hq = 3, 64, 16, 4, 128, 16
+    g = W.rng(5)
+    order = W.free_order(g, N)
+    a = pkv.BlockAllocator(N, B, free_order=order)
+    k_pools = [torch.from_numpy(W.normal_bf16_bits(g, (N, B, Hkv, D)).view(np.int16)).view(torch.bfloat16).cuda()
+               for _ in range(L)]
+    v_pools = [torch.from_numpy(W.normal_bf16_bits(g, (N, B, Hkv, D)).view(np.int16)).view(torch.bfloat16).cuda()
+               for _ in range(L)]
+    n = 300
+    assert a.add_seq(7, n) == 0
+    old = a.table(7)
+    snap_k = [kp[old].clone() for kp in k_pools]
+    snap_v = [vp[old].clone() for vp in v_pools]
+    q = torch.from_numpy(W.normal_bf16_bits(g, (1, Hq, D)).view(np.int16)).view(torch.bfloat16).cuda()
+
+    def attend(table):
+        t = torch.tensor([table], dtype=torch.int32, device="cuda")
+        ln = torch.tensor([n], dtype=torch.int32, device="cuda")
+        return [pkv.paged_decode_attn(q, kp, vp, t, ln, 1 / np.sqrt(D), out_dtype=torch.float32)
+                for kp, vp in zip(k_pools, v_pools)]
+
+    before = attend(old)
+    host = torch.empty(len(old) * L * 2 * B * Hkv * D, dtype=torch.bfloat16).pin_memory()
+    pkv.swap_blocks(k_pools, v_pools, torch.tensor(old, dtype=torch.int32, device="cuda"), host, to_host=True)
+    torch.cuda.synchronize()
+    assert a.free_seq(7) == 0                       # preempted: blocks back to the pool
+    assert a.add_seq(8, N * B) == 0                 # another request takes the whole pool
+    for kp, vp in zip(k_pools, v_pools):
+        kp.fill_(0.0)
+        vp.fill_(0.0)
+    assert a.free_seq(8) == 0
+    assert a.add_seq(7, n) == 0                     # re-admitted: other block ids
+    new = a.table(7)
+    assert new != old
+    pkv.swap_blocks(k_pools, v_pools, torch.tensor(new, dtype=torch.int32, device="cuda"), host, to_host=False)
+    for l in range(L):
+        assert torch.equal(k_pools[l][new].view(torch.int16), snap_k[l].view(torch.int16))
+        assert torch.equal(v_pools[l][new].view(torch.int16), snap_v[l].view(torch.int16))
+    after = attend(new)
+    for x, y in zip(before, after):
+        assert torch.equal(x, y)
+    assert a.check()
+
+
+def test_swap_500mib_time_against_the_pages_estimate():
+    """Move 500 MiB of KV out and back and report the time next to the pages' analytic
+    19.5 ms one way at 25 GiB/s (the measured link may be faster or slower)."""
+    import json
+    import os
+
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    L, B, Hkv, D = 32, 16, 8, 128                    # 128 KiB per token, 2 MiB per block (all layers)
+    nblk = 250                                       # 250 * 2 MiB = 500 MiB
+    N = nblk + 8
+    k_pools = [torch.zeros((N, B, Hkv, D), dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+    v_pools = [torch.zeros((N, B, Hkv, D), dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+    blocks = torch.arange(nblk, dtype=torch.int32, device="cuda")
+    host = torch.empty(nblk * L * 2 * B * Hkv * D, dtype=torch.bfloat16).pin_memory()
+    assert host.numel() * 2 == 500 * 2 ** 20
+    times = {}
+    for name, to_host in (("out", True), ("in", False)):
+        pkv.swap_blocks(k_pools, v_pools, blocks, host, to_host=to_host)     # warm-up
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pkv.swap_blocks(k_pools, v_pools, blocks, host, to_host=to_host)
+        e1.record()
+        torch.cuda.synchronize()
+        times[name] = e0.elapsed_time(e1)
+    rec = {"mib": 500, "out_ms": times["out"], "in_ms": times["in"],
+           "out_gib_per_s": 500 / 1024 / (times["out"] / 1000), "in_gib_per_s": 500 / 1024 / (times["in"] / 1000),
+           "pages_one_way_ms_at_25_gib_per_s": 19.5}
+    os.makedirs("gpurun_out", exist_ok=True)
+    with open("gpurun_out/swap_500mib.json", "w") as f:
+        json.dump(rec, f)
+    assert times["out"] > 0 and times["in"] > 0
