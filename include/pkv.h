@@ -83,13 +83,13 @@ const char* pkv_last_cuda_error(void);
  * attention over the contiguous history up to floating-point rounding: the
  * kernels accumulate in fp32 (products of bf16 inputs are exact in fp32).
  *
- * How: one persistent kernel launch.  All (request, KV-head group, 16-token
- * tile) units are split into equal contiguous ranges, one per CTA; the warps
- * of a CTA take the KV heads of the group over the same tiles, each keeping
- * an online-softmax state (m, l, o) for the grouped query heads of its KV
- * head and reading each K/V tile once per group through a TMA-fed
- * shared-memory ring.  A request split across CTAs is finished by the last
- * CTA to reach it, which merges the partial states
+ * How: one persistent kernel launch of one-warp CTAs (8 per SM; 4 for
+ * 512-byte rows).  All (request, KV head, 16-token tile) units are split into
+ * equal contiguous ranges, one per CTA; the CTA keeps an online-softmax state
+ * (m, l, o) for the grouped query heads of its current KV head and reads each
+ * K/V tile once for the whole group through a TMA-fed shared-memory ring.  A
+ * (request, KV head) split across CTAs is finished by the last CTA to reach
+ * it, which merges the partial states
  * ([P2] exercise "逻辑顺序没错，为什么 attention 输出还是错？": the states merge,
  * per-block outputs do not).
  *
@@ -189,6 +189,35 @@ int pkv_paged_decode_attn_noalloc(const void* q, const void* k_pool, const void*
                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                   int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
                                   int32_t out_dtype, pkv_stream_t stream);
+
+/* Multi-token query: T = num_q_tokens new tokens per request attend at once
+ * (the verification pass of speculative decoding, or a chunk of a prefill),
+ * each under the causal mask inside the last blocks ([P1] section 5: the
+ * staged KV positions of speculative decoding; [P3] section 6 and equation
+ * (4) for each token's attention).  The T tokens are the last T positions of
+ * the history: their K/V must already be in the pools and counted in
+ * seq_lens.  Query token i (0 <= i < T) of request s sits at position
+ * p = seq_lens[s] - T + i and attends positions 0..p:
+ *     out[s][i][h] = sum_{t <= p} softmax_t(scale * <q[s][i][h], K_t>) V_t.
+ * A token with p < 0 (seq_lens[s] < T - i) attends nothing and gets 0.
+ * T = 1 is pkv_paged_decode_attn.
+ *   q, out      [num_seqs][num_q_tokens][num_q_heads][head_dim]
+ *   num_q_tokens 1..16 with G * num_q_tokens <= 16 (G = num_q_heads /
+ *               num_kv_heads): the (query token, grouped head) pairs of a KV
+ *               head share each K/V tile read
+ *   workspace   at least pkv_multi_query_workspace_bytes(...) bytes
+ * Other arguments, layouts and errors as pkv_paged_decode_attn (plans and
+ * runs in one call); pkv_multi_query_workspace_bytes returns 0 for an
+ * unsupported shape. */
+size_t pkv_multi_query_workspace_bytes(int32_t num_seqs, int32_t num_q_tokens, int32_t num_q_heads,
+                                       int32_t num_kv_heads, int32_t head_dim);
+int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                               int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                               pkv_stream_t stream);
 
 /* Synchronises `stream`, reads the workspace status word, clears it and
  * returns PKV_OK, PKV_ERR_BAD_TABLE, PKV_ERR_DEVICE_TIMEOUT or

@@ -96,6 +96,28 @@ def paged_decode(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray,
     return out
 
 
+def multi_query(q: np.ndarray, k_hist: np.ndarray, v_hist: np.ndarray, scale: float) -> np.ndarray:
+    """T query tokens of one request at the last T positions of its history.
+
+    The staged positions of speculative decoding ([P1] "PagedAttention 与在线推理：KV
+    分页、共享及调度的联合分析", section 5) are verified by running every staged
+    token's query at once; each token attends causally, i.e. only up to its own
+    position, with the attention of [P3] section 6.  q: [T, H_q, d];
+    k_hist, v_hist: [n, H_kv, d] holding all n tokens including the T new ones.
+    Token i sits at position p = n - T + i and is dense decode over the first
+    p + 1 tokens; p < 0 (fewer than T - i tokens) attends nothing and gives 0.
+    Returns float64 [T, H_q, d].
+    """
+    T = q.shape[0]
+    n = k_hist.shape[0]
+    out = np.zeros((T,) + q.shape[1:], dtype=np.float64)
+    for i in range(T):
+        p = n - T + i
+        if p >= 0:
+            out[i] = dense_decode(q[i], k_hist[:p + 1], v_hist[:p + 1], scale)
+    return out
+
+
 State = Tuple[np.ndarray, np.ndarray, np.ndarray]  # m [H], l [H], o [H, d]
 
 

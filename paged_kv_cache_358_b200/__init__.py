@@ -18,7 +18,7 @@ __all__ = [
     "lib", "library_path", "Status", "PkvError",
     "BF16", "F32",
     "decode_workspace_bytes", "paged_decode_attn", "decode_plan", "paged_decode_attn_run",
-    "decode_status", "set_decode_kernel", "paged_decode_attn_append_run",
+    "decode_status", "set_decode_kernel", "paged_decode_attn_append_run", "paged_attn_multi_query",
     "kv_append", "block_copy", "slot_mapping", "swap_blocks",
     "BlockAllocator",
 ]
@@ -79,6 +79,9 @@ _SIGS = {
                                                         _vp]),
     "pkv_paged_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                      _i32, _i32, _f32, _i32, _vp, _i32, _vp]),
+    "pkv_multi_query_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "pkv_paged_attn_multi_query": (ctypes.c_int, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                                                  _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
     "pkv_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_ulonglong, _vp, _sz, _vp]),
     "pkv_kv_append": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
@@ -199,6 +202,33 @@ def paged_decode_attn(q, k_pool, v_pool, block_tables, seq_lens, scale: float, o
         _dtype_code(k_pool), _dev(out, "out"), _dtype_code(out), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "paged_decode_attn")
+    return out
+
+
+def paged_attn_multi_query(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out=None,
+                           out_dtype=None, workspace=None, stream=None):
+    """q: [num_seqs, T, num_q_heads, head_dim]; query token i of request s sits at
+    position seq_lens[s] - T + i and attends the paged history up to it (causal)."""
+    torch = _torch()
+    if q.dim() != 4:
+        raise ValueError("q must be [num_seqs, num_q_tokens, num_q_heads, head_dim]")
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have the shape of q")
+    S, T, Hq, D = q.shape
+    _, _, Hkv, _, B, N = _attn_args(q[:, 0], k_pool, v_pool, block_tables, seq_lens, out[:, 0])
+    if workspace is None:
+        n = lib().pkv_multi_query_workspace_bytes(S, T, Hq, Hkv, D)
+        if n == 0:
+            raise PkvError(Status.INVALID, "multi_query_workspace_bytes")
+        workspace = torch.zeros(int(n), dtype=torch.uint8, device=q.device)
+    rc = lib().pkv_paged_attn_multi_query(
+        _dev(q, "q"), T, _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens"), S, Hq, Hkv, D, B, N, float(scale),
+        _dtype_code(k_pool), _dev(out, "out"), _dtype_code(out), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "paged_attn_multi_query")
     return out
 
 

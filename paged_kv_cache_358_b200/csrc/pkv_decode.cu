@@ -217,6 +217,17 @@ bool geometry(int S, int Hq, int Hkv, int D, int dtype, Geometry* g) {
   return true;
 }
 
+// Query heads of the plan for T tokens per request: H_kv * P with P the
+// smallest power of two >= T * G (columns per KV head); 0 if unsupported.
+int32_t multi_query_heads(int32_t T, int32_t Hq, int32_t Hkv) {
+  if (T < 1 || T > 16 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
+  const int cols = T * (Hq / Hkv);
+  if (cols > 16) return 0;
+  int P = 1;
+  while (P < cols) P <<= 1;
+  return Hkv * P;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int do_plan(const Geometry& geo, const int32_t* seq_lens, void* ws, cudaStream_t stream) {
@@ -260,6 +271,13 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
   return best;
 }
 
+size_t pkv_multi_query_workspace_bytes(int32_t num_seqs, int32_t num_q_tokens, int32_t num_q_heads,
+                                       int32_t num_kv_heads, int32_t head_dim) {
+  const int32_t hq_eff = multi_query_heads(num_q_tokens, num_q_heads, num_kv_heads);
+  if (hq_eff <= 0) return 0;
+  return pkv_decode_workspace_bytes(num_seqs, hq_eff, num_kv_heads, head_dim);
+}
+
 int pkv_decode_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
                     int32_t num_kv_heads, int32_t head_dim, int32_t kv_dtype, void* workspace,
                     size_t workspace_bytes, pkv_stream_t stream) {
@@ -276,9 +294,16 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
-             pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots) {
+             pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
+             int32_t num_q_tokens = 1) {
+  // T query tokens per request run as more grouped heads over the same KV
+  // heads: the columns of a KV head are (query token, grouped head), padded
+  // to a power of two.
+  if (new_slots && num_q_tokens != 1) return PKV_ERR_INVALID;
+  const int32_t hq_eff = multi_query_heads(num_q_tokens, num_q_heads, num_kv_heads);
+  if (hq_eff <= 0) return PKV_ERR_INVALID;
   Geometry geo;
-  if (!geometry(num_seqs, num_q_heads, num_kv_heads, head_dim, kv_dtype, &geo)) return PKV_ERR_INVALID;
+  if (!geometry(num_seqs, hq_eff, num_kv_heads, head_dim, kv_dtype, &geo)) return PKV_ERR_INVALID;
   int rc = check_common(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                         block_size, num_blocks, out, out_dtype, workspace, workspace_bytes, geo);
   if (rc != PKV_OK) return rc;
@@ -308,6 +333,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.num_blocks = num_blocks;
   args.out_dtype = out_dtype;
   args.num_workers = geo.NW;
+  args.num_q_tokens = num_q_tokens;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
   args.v_new = new_slots ? v_new : nullptr;
@@ -378,6 +404,29 @@ int pkv_paged_decode_attn(const void* q, const void* k_pool, const void* v_pool,
                                    num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                    num_blocks, scale, kv_dtype, out, out_dtype, workspace,
                                    workspace_bytes, stream);
+}
+
+int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, float scale, int32_t kv_dtype, void* out,
+                               int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                               pkv_stream_t stream) {
+  const int32_t hq_eff = multi_query_heads(num_q_tokens, num_q_heads, num_kv_heads);
+  if (hq_eff <= 0) return PKV_ERR_INVALID;
+  Geometry geo;
+  if (!geometry(num_seqs, hq_eff, num_kv_heads, head_dim, kv_dtype, &geo)) return PKV_ERR_INVALID;
+  int rc = check_common(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                        block_size, num_blocks, out, out_dtype, workspace, workspace_bytes, geo);
+  if (rc != PKV_OK) return rc;
+  if (!std::isfinite(scale)) return PKV_ERR_INVALID;
+  if (num_seqs == 0) return PKV_OK;
+  rc = do_plan(geo, seq_lens, workspace, static_cast<cudaStream_t>(stream));
+  if (rc != PKV_OK) return rc;
+  return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                  num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
+                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, num_q_tokens);
 }
 
 int pkv_decode_status(void* workspace, pkv_stream_t stream) {

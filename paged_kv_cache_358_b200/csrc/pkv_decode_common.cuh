@@ -85,6 +85,7 @@ struct DecodeArgs {
   int32_t block_size, num_blocks;
   int32_t out_dtype;
   int32_t num_workers;
+  int32_t num_q_tokens;  // T query tokens per request (1 for plain decode)
   float scale_log2;     // scale * log2(e)
   // Folded append (all null when the new tokens were appended separately):
   // row s of k_new / v_new is request s's new token, the last of its history,
@@ -114,6 +115,44 @@ PKV_DEVINL long long range_begin(int v, long long T, int NW) {
   return (static_cast<long long>(v) * T) / NW;
 }
 
+// Valid rows of a tile for each column of the grouped computation.  A column
+// is (query token i, grouped head k), c = i * Gq + k.  With T query tokens per
+// request at the last T positions, token i sees positions < len - (T-1-i)
+// (causal); rows at or past the length hold no data at all.  Single-token
+// decode (kCausal = false) masks by the length alone, with no per-column work.
+template <bool kCausal>
+struct TileLim {
+  static constexpr bool causal = kCausal;  // columns may differ, and may see no row
+  int nvalid;  // rows holding tokens of the request (1..16)
+  int rem;     // length - first position of the tile (may exceed 16)
+  int T;       // query tokens per request
+  int Gq;      // grouped query heads per KV head
+  PKV_DEVINL int lim(int c) const {
+    if constexpr (!kCausal) {
+      return nvalid;
+    } else {
+      const int causal_lim = rem - (T - 1 - c / Gq);
+      return causal_lim < nvalid ? causal_lim : nvalid;
+    }
+  }
+};
+
+// Output row of column c: out[s][i][head * Gq + k][:] for c = i * Gq + k,
+// given the row of column 0 and the stride between query tokens (H_q * d).
+// Columns c >= ncols (= T * Gq, padded up to the kernel's power-of-two group)
+// are not written.
+struct OutMap {
+  size_t row0;
+  size_t tok_stride;
+  int Gq;
+  int D;
+  int ncols;
+  PKV_DEVINL size_t row(int c) const {
+    if (ncols == Gq) return row0 + static_cast<size_t>(c) * D;  // one token: rows are adjacent
+    return row0 + static_cast<size_t>(c / Gq) * tok_stride + static_cast<size_t>(c % Gq) * D;
+  }
+};
+
 // Per-stage metadata written by the issuing lane, read by the consuming warp.
 struct alignas(16) StageMeta {
   int32_t s;       // request
@@ -123,7 +162,8 @@ struct alignas(16) StageMeta {
                    // tile; bits 8..: valid tokens in the tile
   int32_t nt;      // tiles of the pair
   int32_t new_slot;  // folded append: pool slot of the pair's new token (< 0: none)
-  int32_t pad[2];
+  int32_t len;       // length of the request
+  int32_t pad;
 };
 
 }  // namespace pkv

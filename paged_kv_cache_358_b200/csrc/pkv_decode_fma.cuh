@@ -96,8 +96,10 @@ struct FmaCore {
     st.l = 0.f;
   }
 
-  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, int nvalid,
+  template <class Lim>
+  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, const Lim& L,
                               float* scratch, int lane) {
+    const int nvalid = L.nvalid;
     const int u = lane & (U - 1);
     const int tg = lane >> LOGU;
     float* sbuf = scratch;               // [kTile][G] scores, then p
@@ -142,7 +144,7 @@ struct FmaCore {
       const int idx = hb * NF + i;
       const int k = idx / R, r = idx % R;
       const int t = tg * R + r;
-      const float s = t < nvalid ? X[i] : -INFINITY;
+      const float s = t < L.lim(k) ? X[i] : -INFINITY;
       if (owner) sbuf[t * G + k] = s;
     }
     __syncwarp();
@@ -160,11 +162,14 @@ struct FmaCore {
 #pragma unroll
     for (int msk = 1; msk < LPH; msk <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, msk));
     const float m_new = fmaxf(st.m, mt);
-    const float alpha = exp2f(st.m - m_new);
+    // no valid score yet for this head: subtract 0 so every exponent is 0, not NaN
+    float m_ref = m_new;
+    if constexpr (Lim::causal) m_ref = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = exp2f(st.m - m_ref);
     float psum = 0.f;
 #pragma unroll
     for (int i = 0; i < TPL; ++i) {
-      const float p = exp2f(sv[i] - m_new);
+      const float p = exp2f(sv[i] - m_ref);
       psum += p;
       if (active) sbuf[(li * TPL + i) * G + kh] = p;
     }
@@ -221,7 +226,7 @@ struct FmaCore {
   // Reduce the warp's state and write either the final output (complete
   // pair) or a partial state (o[G][D], m[G], l[G]) for the merge kernel.
   static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype,
-                                size_t out_row /* (s*H_q + g*G) * D */, float* part, int lane) {
+                                const OutMap& om, float* part, int lane) {
     const int u = lane & (U - 1);
     const int tg = lane >> LOGU;
 #pragma unroll
@@ -243,11 +248,11 @@ struct FmaCore {
       if (tg == 0) {
 #pragma unroll
         for (int k = 0; k < G; ++k) {
-          const float inv = 1.f / lk[k];
+          const float inv = lk[k] > 0.f ? 1.f / lk[k] : 0.f;  // 0: nothing attended
           float v[E];
 #pragma unroll
           for (int e = 0; e < E; ++e) v[e] = st.o[k][e] * inv;
-          store_out(out, out_dtype, out_row + size_t(k) * D + size_t(u) * E, v);
+          if (k < om.ncols) store_out(out, out_dtype, om.row(k) + size_t(u) * E, v);
         }
       }
     } else {

@@ -24,9 +24,9 @@ namespace pkv {
 // ---------------------------------------------------------------------------
 // Kept out of line: its load batches need many registers for a moment, and
 // inlined they would raise the register count of the whole streaming loop.
-template <int D, int G, int HG>
+template <int D, int G, int HG, bool MULTI>
 __device__ __noinline__ void merge_pair(const float* partials, long long pp, int w, int v0, int v1, long long T,
-                           int NW, void* out, int out_dtype, size_t out_row, int lane) {
+                           int NW, void* out, int out_dtype, OutMap om, int lane) {
   constexpr int PS = part_stride(G, D);
   constexpr int PER = D / 32;   // output elements per lane
   constexpr int UMAX = 32 / G;  // CTAs per pass: lane i reads (CTA i / G, head i % G)
@@ -64,8 +64,11 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
 #pragma unroll
     for (int msk = G; msk < 32; msk <<= 1) mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, msk));
     const float nm = fmaxf(run_m, mk);
-    const float old_scale = exp2f(run_m - nm);  // 0 on the first pass
-    const float wgt = valid ? exp2f(mv - nm) : 0.f;
+    // under the causal mask a column no CTA saw a token for keeps m = -inf:
+    // subtract 0 there, not -inf
+    const float nms = (MULTI && nm == -INFINITY) ? 0.f : nm;
+    const float old_scale = exp2f(run_m - nms);  // 0 on the first pass
+    const float wgt = valid ? exp2f(mv - nms) : 0.f;
     float wl = wgt * lv;
 #pragma unroll
     for (int msk = G; msk < 32; msk <<= 1) wl += __shfl_xor_sync(0xffffffffu, wl, msk);
@@ -99,17 +102,25 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
   }
 #pragma unroll
   for (int k = 0; k < G; ++k) {
-    const float inv = 1.f / __shfl_sync(0xffffffffu, run_l, k);
+    const float lk = __shfl_sync(0xffffffffu, run_l, k);
+    if constexpr (MULTI) {
+      const float inv = lk > 0.f ? 1.f / lk : 0.f;  // a column with no visible token is 0
+      if (k < om.ncols)
 #pragma unroll
-    for (int i = 0; i < PER; ++i) store1(out, out_dtype, out_row + k * D + lane * PER + i, acc[k][i] * inv);
+        for (int i = 0; i < PER; ++i) store1(out, out_dtype, om.row(k) + lane * PER + i, acc[k][i] * inv);
+    } else {
+      const float inv = 1.f / lk;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) store1(out, out_dtype, om.row0 + k * D + lane * PER + i, acc[k][i] * inv);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Partition: persistent grid, one stream-K worker per CTA, one KV head per warp.
 // ---------------------------------------------------------------------------
-// One lookahead entry: s, hg | nt << 12, j, flags, new_slot, phys[kMaxBoxes].
-constexpr int kEntryInts = 5 + kMaxBoxes;
+// One lookahead entry: s, hg | nt << 12, j, flags, new_slot, len, phys[kMaxBoxes].
+constexpr int kEntryInts = 6 + kMaxBoxes;
 
 template <class Core, int W, int DEPTH>
 struct Smem {
@@ -142,7 +153,10 @@ struct TmaMaps {
   CUtensorMap v;
 };
 
-template <class Core, int G, int W, int CPS, int DEPTH>
+// MULTI: several query tokens per request (causal) or idle padding columns;
+// without it the columns are exactly the G grouped heads of one token and the
+// kernel has no per-column work.
+template <class Core, int G, int W, int CPS, int DEPTH, bool MULTI>
 __global__ void __launch_bounds__(W * 32, CPS)
     partition_kernel(const __grid_constant__ TmaMaps maps, const DecodeArgs a, int check_S,
                      int check_Hq, int check_Hkv, int check_D, int check_dtype) {
@@ -168,7 +182,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
     if (threadIdx.x == 0) record_status(status, kStatusPlanMismatch);
     return;
   }
-  const long long T = hdr->total_tiles;
+  const long long TT = hdr->total_tiles;
   const int NW = a.num_workers;
   const int v = blockIdx.x;  // this CTA's worker id; warp = head within the group
   const int4 wp = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[2 * v];
@@ -177,12 +191,24 @@ __global__ void __launch_bounds__(W * 32, CPS)
 
   const int S = a.num_seqs, Hkv = a.num_kv_heads, NHG = a.head_groups, Bsz = a.block_size;
   const int Hq = a.num_q_heads;
+  // T query tokens per request: the columns of a KV head are its Gq grouped
+  // heads for each token, c = i * Gq + k, padded with idle columns up to G.
+  const int T = MULTI ? a.num_q_tokens : 1;
+  const int Gq = MULTI ? Hq / Hkv : G;
+  const int ncols = MULTI ? T * Gq : G;
   const int box_rows = Bsz < kTile ? Bsz : kTile;
   const int nbox = kTile / box_rows;  // boxes per tile per chunk
   const uint64_t pol = policy_evict_first();
   float* partials = reinterpret_cast<float*>(a.ws + a.off_partials);
   int32_t* counters = reinterpret_cast<int32_t*>(a.ws + a.off_counters);
 
+  if (ntiles > 0 && ncols < G) {
+    // idle columns read zeros: the bulk copies fill only the first ncols q rows
+    for (int st = 0; st < DEPTH; ++st)
+      for (int i = ncols * Core::ROWB / 16 + lane; i < Core::QB / 16; i += 32)
+        reinterpret_cast<uint4*>(stages + st * Core::kStageBytes + Core::kQOff)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   if (ntiles > 0 && lane == 0) {
     for (int i = 0; i < DEPTH; ++i) mbar_init(smem_u32(&bars[i]), 1);
     fence_mbar_init();
@@ -197,7 +223,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
   // read when the walk crosses into a new request.
   int cs = wp.z, coff = wp.w;
   int clen = first_len;
-  int n_s = 0, n_hg = 0, n_j = 0, n_flags = 0, n_nt = 0;
+  int n_s = 0, n_hg = 0, n_j = 0, n_flags = 0, n_nt = 0, n_len = 0;
   long long n_slot = -1;
   int n_phys[kMaxBoxes];
   uint32_t n_have = 0, n_over = 0;  // bit b: box b is read / box b lies past the table row
@@ -230,6 +256,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       n_j = j;
       n_nt = nt;
       n_flags = (min(kTile, len - j * kTile) << 8) | (j == nt - 1 ? 2 : 0);
+      n_len = len;
       n_slot = (a.new_slots != nullptr && j == nt - 1) ? a.new_slots[s] : -1;
       const int32_t* row = a.block_tables + static_cast<size_t>(s) * a.max_blocks;
 #pragma unroll
@@ -266,6 +293,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
         record_status(status, kStatusBadTable);  // new-token slot outside the pool: not written
       else if (n_slot >= 0)
         e[4] = static_cast<int>(n_slot);
+      if constexpr (MULTI) e[5] = n_len;
 #pragma unroll
       for (int b = 0; b < kMaxBoxes; ++b) {
         int phys = -1;
@@ -278,7 +306,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
             phys = a.num_blocks;  // out of the tensor map: TMA fills zeros
           }
         }
-        e[5 + b] = phys;
+        e[6 + b] = phys;
       }
     }
     __syncwarp();
@@ -305,24 +333,28 @@ __global__ void __launch_bounds__(W * 32, CPS)
       meta[st].flags = e[3] | (newpair ? 1 : 0);
       meta[st].nt = e[1] >> 12;
       meta[st].new_slot = e[4];
+      if constexpr (MULTI) meta[st].len = e[5];
       const uint32_t bar = smem_u32(&bars[st]);
       int nb = 0;
 #pragma unroll
-      for (int b = 0; b < kMaxBoxes; ++b) nb += (b < nbox && e[5 + b] >= 0) ? 1 : 0;
+      for (int b = 0; b < kMaxBoxes; ++b) nb += (b < nbox && e[6 + b] >= 0) ? 1 : 0;
       const uint32_t box_bytes = static_cast<uint32_t>(box_rows * Core::kChunkRowBytes);
       uint32_t bytes = 2u * nb * Core::kChunks * box_bytes;
-      if (newpair) bytes += Core::QB;
+      if (newpair) bytes += ncols * Core::ROWB;
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(bar, bytes);
       if (newpair) {
-        const char* qsrc = reinterpret_cast<const char*>(a.q) +
-                           (static_cast<size_t>(s) * Hq + static_cast<size_t>(head) * G) * Core::ROWB;
-        bulk_load(smem_u32(stage + Core::kQOff), qsrc, Core::QB, bar);
+        // the pair's G columns: Gq grouped heads of each of the T query tokens
+        for (int i = 0; i < T; ++i) {
+          const char* qsrc = reinterpret_cast<const char*>(a.q) +
+                             ((static_cast<size_t>(s) * T + i) * Hq + static_cast<size_t>(head) * Gq) * Core::ROWB;
+          bulk_load(smem_u32(stage + Core::kQOff + i * Gq * Core::ROWB), qsrc, Gq * Core::ROWB, bar);
+        }
       }
       const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
 #pragma unroll
       for (int b = 0; b < kMaxBoxes; ++b) {
-        const int phys = e[5 + b];
+        const int phys = e[6 + b];
         if (b < nbox && phys >= 0) {
 #pragma unroll
           for (int c = 0; c < Core::kChunks; ++c) {
@@ -348,8 +380,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
   for (long long p = v; p < static_cast<long long>(S) * NHG; p += NW) {
     const int s = static_cast<int>(p / NHG), hg = static_cast<int>(p % NHG);
     if (a.seq_lens[s] != 0) continue;
-    const size_t row = (static_cast<size_t>(s) * Hq + static_cast<size_t>(hg * W + warp) * G) * D;
-    for (int i = lane; i < G * D; i += 32) store1(a.out, a.out_dtype, row + i, 0.f);
+    const OutMap om{(static_cast<size_t>(s) * T * Hq + static_cast<size_t>(hg * W + warp) * Gq) * D,
+                    static_cast<size_t>(Hq) * D, Gq, D, ncols};
+    for (int i = lane; i < ncols * D; i += 32) store1(a.out, a.out_dtype, om.row(i / D) + i % D, 0.f);
   }
   if (ntiles <= 0) return;
 
@@ -361,14 +394,15 @@ __global__ void __launch_bounds__(W * 32, CPS)
 
   auto flush = [&]() {
     const int head = phg * W + warp;
-    const size_t out_row = (static_cast<size_t>(ps) * Hq + static_cast<size_t>(head) * G) * D;
+    const OutMap om{(static_cast<size_t>(ps) * T * Hq + static_cast<size_t>(head) * Gq) * D,
+                    static_cast<size_t>(Hq) * D, Gq, D, ncols};
     if (jfirst == 0 && last_is_end) {  // the whole pair is in this CTA's range
-      Core::finish(state, true, a.out, a.out_dtype, out_row, nullptr, lane);
+      Core::finish(state, true, a.out, a.out_dtype, om, nullptr, lane);
       return;
     }
     const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
     float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
-    Core::finish(state, false, a.out, a.out_dtype, out_row, part, lane);
+    Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
     // Count this CTA in for (request, KV head); the last CTA of the pair merges.
     const size_t ctr = static_cast<size_t>(ps) * Hkv + head;
     // Release the warp's partial writes and count in (acquire-release at GPU
@@ -377,15 +411,15 @@ __global__ void __launch_bounds__(W * 32, CPS)
     int prev = 0;
     if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[ctr], 1);
     prev = __shfl_sync(0xffffffffu, prev, 0);
-    const int v0 = owner_of(pstart, T, NW), v1 = owner_of(pstart + pnt - 1, T, NW);
-    int expected = v1 - v0 + 1;  // with T >= NW every CTA owns at least one tile
-    if (T < NW) {
+    const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + pnt - 1, TT, NW);
+    int expected = v1 - v0 + 1;  // with TT >= NW every CTA owns at least one tile
+    if (TT < NW) {
       expected = 0;
-      for (int u = v0; u <= v1; ++u) expected += range_begin(u, T, NW) < range_begin(u + 1, T, NW) ? 1 : 0;
+      for (int u = v0; u <= v1; ++u) expected += range_begin(u, TT, NW) < range_begin(u + 1, TT, NW) ? 1 : 0;
     }
     if (prev == expected - 1) {
       __syncwarp();  // lane 0's acquire orders the whole warp's loads (barrier semantics)
-      merge_pair<D, G, W>(partials, pp, warp, v0, v1, T, NW, a.out, a.out_dtype, out_row, lane);
+      merge_pair<D, G, W, MULTI>(partials, pp, warp, v0, v1, TT, NW, a.out, a.out_dtype, om, lane);
       if (lane == 0) atomicExch(&counters[ctr], 0);
     }
   };
@@ -428,10 +462,11 @@ __global__ void __launch_bounds__(W * 32, CPS)
       }
       __syncwarp();
     }
+    const TileLim<MULTI> lim{nvalid, MULTI ? m.len - m.j * kTile : nvalid, T, Gq};
     if constexpr (Core::kSwizzle) {
-      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, nvalid, a.scale_log2, lane);
+      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, lim, a.scale_log2, lane);
     } else {
-      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, nvalid, scratch, lane);
+      Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, lim, scratch, lane);
     }
     __syncwarp();
     if (k + DEPTH < ntiles) issue(k + DEPTH);
@@ -454,7 +489,7 @@ extern int g_kernel_choice;  // 0 auto, 1 CUDA-core tiles, 2 tensor-core tiles (
 bool make_pool_map(CUtensorMap* m, const void* pool, int dtype, int D, int B, int Hkv, int N,
                    int box_inner, int box_rows, bool swizzle);
 
-template <class Core, int G, int W, int CPS>
+template <class Core, int G, int W, int CPS, bool MULTI>
 int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_pool, const void* v_pool,
                      cudaStream_t stream) {
   constexpr int DEPTH = pick_depth<Core, W, CPS>();
@@ -469,7 +504,7 @@ int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_
     host::set_error("cuTensorMapEncodeTiled failed");
     return PKV_ERR_CUDA;
   }
-  auto kern = partition_kernel<Core, G, W, CPS, DEPTH>;
+  auto kern = partition_kernel<Core, G, W, CPS, DEPTH, MULTI>;
   static thread_local int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -487,7 +522,9 @@ int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, cons
                 cudaStream_t stream) {
   constexpr int WPS = (Core::ROWB >= 512) ? 4 : 8;
   if (geo.HG != 1) return PKV_ERR_INVALID;
-  return launch_partition<Core, G, 1, WPS>(geo, args, k, v, stream);
+  if (args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads)
+    return launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream);
+  return launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
 }
 
 // One (storage type, head_dim): dispatch on the group size and the core.

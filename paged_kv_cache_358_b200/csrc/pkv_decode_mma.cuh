@@ -117,8 +117,10 @@ struct MmaCore {
     st.l[0] = st.l[1] = 0.f;
   }
 
-  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, int nvalid, float scale_log2,
-                              int lane) {
+  template <class Lim>
+  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, const Lim& L,
+                              float scale_log2, int lane) {
+    const int nvalid = L.nvalid;
     const int gid = lane >> 2, tig = lane & 3;
     const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
 
@@ -134,12 +136,13 @@ struct MmaCore {
         mma_bf16_16816(c, a0, a1, a2, a3, st.qb[kk][0], st.qb[kk][1]);
       }
     }
-    // c[0]: (tok gid, head 2tig), c[1]: (gid, 2tig+1), c[2]: (gid+8, 2tig), c[3]: (gid+8, 2tig+1)
+    // c[0]: (tok gid, col 2tig), c[1]: (gid, 2tig+1), c[2]: (gid+8, 2tig), c[3]: (gid+8, 2tig+1)
+    const int lim0 = L.lim(2 * tig), lim1 = L.lim(2 * tig + 1);
     float s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = gid + ((i & 2) ? 8 : 0);
-      s[i] = t < nvalid ? c[i] * scale_log2 : -INFINITY;
+      s[i] = t < ((i & 1) ? lim1 : lim0) ? c[i] * scale_log2 : -INFINITY;
     }
     float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
 #pragma unroll
@@ -148,11 +151,19 @@ struct MmaCore {
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
     }
     const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
-    const float al0 = exp2f(st.m[0] - mn0), al1 = exp2f(st.m[1] - mn1);
+    // Under the causal mask a column may have seen no valid score yet and keep
+    // m = -inf: subtract 0 instead, so every exponent is exp2(-inf) = 0 and
+    // nothing becomes NaN.  Without it every tile has a valid row.
+    float r0 = mn0, r1 = mn1;
+    if constexpr (Lim::causal) {
+      r0 = mn0 == -INFINITY ? 0.f : mn0;
+      r1 = mn1 == -INFINITY ? 0.f : mn1;
+    }
+    const float al0 = exp2f(st.m[0] - r0), al1 = exp2f(st.m[1] - r1);
     st.m[0] = mn0;
     st.m[1] = mn1;
-    const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
-    const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
+    const float p0 = exp2f(s[0] - r0), p1 = exp2f(s[1] - r1);
+    const float p2 = exp2f(s[2] - r0), p3 = exp2f(s[3] - r1);
     st.l[0] = st.l[0] * al0 + (p0 + p2);
     st.l[1] = st.l[1] * al1 + (p1 + p3);
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
@@ -191,7 +202,7 @@ struct MmaCore {
     }
   }
 
-  static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, size_t out_row,
+  static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, const OutMap& om,
                                 float* part, int lane) {
     const int gid = lane >> 2, tig = lane & 3;
     float l0 = st.l[0], l1 = st.l[1];
@@ -202,17 +213,18 @@ struct MmaCore {
     }
     const int h0 = 2 * tig, h1 = 2 * tig + 1;
     if (complete) {
-      const float i0 = 1.f / l0, i1 = 1.f / l1;
+      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;  // 0: nothing attended
+      const size_t r0 = om.row(h0), r1 = om.row(h1);
 #pragma unroll
       for (int mt = 0; mt < KSTEPS; ++mt) {
         const int d0 = 16 * mt + gid, d1 = d0 + 8;
-        if (h0 < G) {
-          put(out, out_dtype, out_row + size_t(h0) * D + d0, st.oc[mt][0] * i0);
-          put(out, out_dtype, out_row + size_t(h0) * D + d1, st.oc[mt][2] * i0);
+        if (h0 < om.ncols) {
+          put(out, out_dtype, r0 + d0, st.oc[mt][0] * i0);
+          put(out, out_dtype, r0 + d1, st.oc[mt][2] * i0);
         }
-        if (h1 < G) {
-          put(out, out_dtype, out_row + size_t(h1) * D + d0, st.oc[mt][1] * i1);
-          put(out, out_dtype, out_row + size_t(h1) * D + d1, st.oc[mt][3] * i1);
+        if (h1 < om.ncols) {
+          put(out, out_dtype, r1 + d0, st.oc[mt][1] * i1);
+          put(out, out_dtype, r1 + d1, st.oc[mt][3] * i1);
         }
       }
     } else {

@@ -194,3 +194,62 @@ def test_extreme_logits_stay_finite(qscale):
     assert np.max(np.abs(dense - ref)) < 1e-12
     online = att.online_decode_blocks(q, K, V, scale, 16)
     assert np.max(np.abs(online - dense)) < 1e-12
+
+
+# -- multi-token query --------------------------------------------------------
+def _sdpa_causal_tail_f64(q, K, V, scale):
+    """q [T, H_q, d] at the last T of n positions, K/V [n, H_kv, d] -> [T, H_q, d]
+    through torch SDPA with an explicit bottom-right causal mask (n >= T)."""
+    T, H_q, _ = q.shape
+    n, H_kv, _ = K.shape
+    G = H_q // H_kv
+    qt = torch.from_numpy(q).permute(1, 0, 2)                               # [H_q, T, d]
+    kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(G, dim=0)   # [H_q, n, d]
+    vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(G, dim=0)
+    pos = torch.arange(n)[None, :]
+    mask = pos <= (n - T + torch.arange(T))[:, None]                        # [T, n]
+    out = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None],
+                                                           attn_mask=mask, scale=scale)
+    return out[0].permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("n,T,H_q,H_kv,d", [(9, 3, 8, 2, 16), (40, 4, 4, 4, 32), (5, 5, 2, 1, 8),
+                                            (100, 8, 16, 8, 64), (17, 16, 1, 1, 16)])
+def test_multi_query_matches_torch_causal_sdpa(n, T, H_q, H_kv, d):
+    g = rng(300 + n + T)
+    q = normal_f32(g, (T, H_q, d)).astype(np.float64)
+    K = normal_f32(g, (n, H_kv, d)).astype(np.float64)
+    V = normal_f32(g, (n, H_kv, d)).astype(np.float64)
+    scale = 1.0 / np.sqrt(d)
+    ref = _sdpa_causal_tail_f64(q, K, V, scale)
+    out = att.multi_query(q, K, V, scale)
+    assert np.max(np.abs(out - ref)) < 1e-13
+
+
+def test_multi_query_special_cases():
+    g = rng(7)
+    T, H_q, H_kv, d = 4, 4, 2, 16
+    q = normal_bf16_bits(g, (T, H_q, d))
+    K = normal_bf16_bits(g, (6, H_kv, d))
+    V = normal_bf16_bits(g, (6, H_kv, d))
+    # one token: plain decode over the whole history
+    one = att.multi_query(q[:1], K, V, 0.25)
+    assert np.array_equal(one[0], att.dense_decode(q[0], K, V, 0.25))
+    # the last token sees everything; token 0 of a history of T tokens sees only token 0 -> v_0
+    out = att.multi_query(q, K[:T], V[:T], 0.25)
+    assert np.array_equal(out[-1], att.dense_decode(q[-1], K[:T], V[:T], 0.25))
+    Vf = att.widen(V)
+    for h in range(H_q):
+        assert np.array_equal(out[0, h], Vf[0, h // (H_q // H_kv)])
+    # fewer tokens than queries: tokens before the history's start give 0
+    short = att.multi_query(q, K[:2], V[:2], 0.25)
+    assert not short[:2].any()
+    assert np.array_equal(short[2, 0], Vf[0, 0])
+    # causality: poisoning the positions after token i leaves row i unchanged
+    Kp, Vp = att.widen(K).copy(), att.widen(V).copy()
+    Kp[4:] = np.nan
+    Vp[4:] = np.nan
+    pois = att.multi_query(q, Kp, Vp, 0.25)
+    clean = att.multi_query(q, K, V, 0.25)
+    assert np.array_equal(pois[:2], clean[:2])      # tokens at positions 2, 3
+    assert np.isnan(pois[2:]).all()

@@ -168,3 +168,27 @@ def test_copy_length_mutant_is_caught():
         good = copies == [(a.table(1)[1], a.table(0)[1], 3)] and a.table(0)[0] == a.table(1)[0] \
             and a.ref[a.table(0)[0]] == 2
         assert good == expect_ok
+
+
+# -- multi-token query mutant -------------------------------------------------
+def _multi_query_off_by_one(q, k_hist, v_hist, scale):
+    T, n = q.shape[0], k_hist.shape[0]
+    out = np.zeros((T,) + q.shape[1:])
+    for i in range(T):
+        p = n - T + i
+        if p >= 0:       # sees one token past its own position
+            out[i] = att.dense_decode(q[i], k_hist[:p + 2], v_hist[:p + 2], scale)
+    return out
+
+
+MQ_PINS = [lambda: TA.test_multi_query_matches_torch_causal_sdpa(9, 3, 8, 2, 16),
+           TA.test_multi_query_special_cases]
+
+
+def test_unmutated_multi_query_passes_pins():
+    assert not _any_pin_fails(MQ_PINS)
+
+
+def test_multi_query_mutant_is_caught(monkeypatch):
+    monkeypatch.setattr(att, "multi_query", _multi_query_off_by_one)
+    assert _any_pin_fails(MQ_PINS)
