@@ -61,6 +61,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
+    p.add_argument("--no-extras", action="store_true", help="skip the swap and allocator measurements")
     p.add_argument("--unfused", action="store_true",
                    help="append with a separate kv_append launch instead of folding it into attention")
     p.add_argument("--layers", type=int, default=32,
@@ -373,31 +374,97 @@ def _blas_threads():
 def cpu_baseline(seconds: float):
     """The float64 oracle, as it stands, on a bounded sample of the same workload.
 
-    Requests of the 32 x 4096 batch are drawn and attended one at a time (one
-    layer) until `seconds` of oracle compute have been spent; input generation
-    is not timed.
+    The 32 request histories (4096 tokens) are drawn once; layer after layer,
+    a fresh q is drawn and each request is attended one at a time until
+    `seconds` of oracle compute have been spent.  Input generation is not
+    timed.
     """
     import workloads as W
     from oracle import attention as oatt
 
     wl = W.workload("teaching_32x4096")
     g = W.rng(123)
-    compute, done_bytes, n_req = 0.0, 0, 0
-    while compute < seconds and n_req < wl.num_seqs:
-        n = wl.lengths[n_req]
-        kh = W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim))
-        vh = W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim))
-        q = W.normal_bf16_bits(g, (wl.num_q_heads, wl.head_dim))
-        t1 = time.perf_counter()
-        oatt.dense_decode(q, kh, vh, wl.scale)
-        compute += time.perf_counter() - t1
-        done_bytes += n * wl.num_kv_heads * wl.head_dim * 2 * 2 + 2 * wl.num_q_heads * wl.head_dim * 2
-        n_req += 1
+    hist = [(W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim)),
+             W.normal_bf16_bits(g, (n, wl.num_kv_heads, wl.head_dim))) for n in wl.lengths]
+    compute, done_bytes, n_att, layers = 0.0, 0, 0, 0
+    while compute < seconds and layers < wl.layers:
+        for s, n in enumerate(wl.lengths):
+            q = W.normal_bf16_bits(g, (wl.num_q_heads, wl.head_dim))
+            t1 = time.perf_counter()
+            oatt.dense_decode(q, hist[s][0], hist[s][1], wl.scale)
+            compute += time.perf_counter() - t1
+            done_bytes += n * wl.num_kv_heads * wl.head_dim * 2 * 2 + 2 * wl.num_q_heads * wl.head_dim * 2
+            n_att += 1
+            if compute >= seconds:
+                break
+        layers += 1
     return {"value": done_bytes / compute / 1e9, "unit": "GB/s", "cores": _blas_threads(),
             "host_cpus": os.cpu_count(), "kind": "oracle",
-            "sample": f"float64 NumPy dense decode attention of {n_req} of the 32 requests x 4096 "
-                      f"history, one layer (H_q 32, H_kv 8, d 128); {compute:.1f} s of CPU work, "
+            "sample": f"float64 NumPy dense decode attention of {n_att} (request, layer) pairs of the "
+                      f"32 requests x 4096 history (H_q 32, H_kv 8, d 128; histories drawn once and "
+                      f"reused across {layers} layers, fresh q per layer); {compute:.1f} s of CPU work, "
                       f"input generation not timed"}
+
+
+def swap_measurement():
+    """Preemption by swap: move 500 MiB of KV (250 blocks of the teaching model,
+    32 layers, K and V) to pinned host memory and back; the pages estimate
+    19.5 ms one way at 25 GiB/s."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    L, B, Hkv, D, nblk = 32, 16, 8, 128, 250
+    kp = [torch.zeros((nblk + 4, B, Hkv, D), dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+    vp = [torch.zeros_like(kp[0]) for _ in range(L)]
+    blocks = torch.arange(nblk, dtype=torch.int32, device="cuda")
+    host = torch.empty(nblk * L * 2 * B * Hkv * D, dtype=torch.bfloat16).pin_memory()
+    res = {"mib": host.numel() * 2 / 2**20, "pages_one_way_ms_at_25_gib_per_s": 19.5}
+    for name, to_host in (("out", True), ("in", False)):
+        pkv.swap_blocks(kp, vp, blocks, host, to_host=to_host)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pkv.swap_blocks(kp, vp, blocks, host, to_host=to_host)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        res[f"{name}_ms"] = ms
+        res[f"{name}_gib_per_s"] = res["mib"] / 1024 / (ms / 1000)
+    del kp, vp, host
+    return res
+
+
+def allocator_measurement(seconds: float = 1.0):
+    """Host allocator throughput (C++): admit with prefix-cache hits, decode
+    appends, release, on a 4096-block pool; operations per second."""
+    import paged_kv_cache_358_b200 as pkv
+
+    a = pkv.BlockAllocator(4096, 16, enable_cache=True)
+    ids = np.arange(64, dtype=np.int32)
+    st = np.zeros(64, dtype=np.int32)
+    cp = np.zeros((64, 3), dtype=np.int32)
+    ops = 0
+    t0 = time.perf_counter()
+    rnd = 0
+    while time.perf_counter() - t0 < seconds:
+        for i in ids:
+            keys = [(int(i) % 8) * 100 + k for k in range(4)]
+            rc, _ = a.add_seq_prefix(int(i), 64 + int(i) % 16, keys)
+            if rc == 0:
+                for k in range(4):
+                    a.set_block_key(int(i), k, keys[k])
+        for _ in range(16):
+            a.append_arrays(ids, st, cp)
+        for i in ids:
+            a.free_seq(int(i))
+        ops += 64 * 2 + 16 * 64 + 64 * 4
+        rnd += 1
+    dt = time.perf_counter() - t0
+    assert a.check()
+    return {"ops_per_s": ops / dt, "note": "admit with prefix hits + 4 key registrations + 16 appends + release, "
+                                             "per request, 64 requests per round, through the Python binding",
+            "prefix_hits": a.stats()["prefix_hits"]}
 
 
 def reference_arm(args):
@@ -503,6 +570,9 @@ def main():
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             cpu = cpu_baseline(args.cpu_seconds)
+        extras = None
+        if world == 1 and not args.no_extras:
+            extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement()}
         steps_per_s = args.steps / (ms_max / 1000) * world
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -527,6 +597,7 @@ def main():
             "cpu_baseline": cpu,
             "clocks": clk,
             "gpu_launches": launches,
+            "extras": extras,
             "wall_s_timed": wall,
         }
         print(json.dumps(result), flush=True)
