@@ -435,6 +435,53 @@ def swap_measurement():
     return res
 
 
+def multi_query_measurement(reps: int = 20):
+    """Multi-token query (T tokens per request, causal) on one layer of the
+    32 x 4096 teaching shapes: microseconds per call (plan + attention) and
+    algorithmic GB/s (history K/V once per KV head, q and out of all T tokens,
+    tables), for T = 1, 2, 4.  Pools hold 12 layers' worth of blocks and the
+    calls rotate over them, so every call streams from HBM."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    import workloads as W
+
+    wl = W.workload("teaching_32x4096", decode_steps=16)
+    S, Hq, Hkv, D, B, N = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.pool_blocks
+    a = pkv.BlockAllocator(N, B, free_order=W.free_order(W.rng(5), N))
+    for i, n in enumerate(wl.lengths):
+        assert a.add_seq(i, n) == 0
+    tables, lens = a.fill_tables(list(range(S)), -(-max(wl.lengths) // B))
+    td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    copies = 12
+    kp = [torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
+    vp = [torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
+    res = {}
+    for T in (1, 2, 4):
+        q = torch.randn((S, T, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
+        out = torch.empty_like(q)
+        ws = torch.zeros(pkv.lib().pkv_multi_query_workspace_bytes(S, T, Hq, Hkv, D), dtype=torch.uint8,
+                         device="cuda")
+        for i in range(3):
+            pkv.paged_attn_multi_query(q, kp[i], vp[i], td, ld, wl.scale, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(reps):
+            pkv.paged_attn_multi_query(q, kp[i % copies], vp[i % copies], td, ld, wl.scale, out=out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000 / reps
+        nbytes = (int(lens.sum()) * Hkv * D * 2 * 2 + 2 * S * T * Hq * D * 2
+                  + 4 * int(sum(-(-int(n) // B) for n in lens)) + 4 * S)
+        res[f"T{T}"] = {"us_per_call": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9,
+                        "columns_per_kv_head": T * Hq // Hkv}
+    del kp, vp
+    return res
+
+
 def allocator_measurement(seconds: float = 1.0):
     """Host allocator throughput (C++): admit with prefix-cache hits, decode
     appends, release, on a 4096-block pool; operations per second."""
@@ -572,7 +619,8 @@ def main():
             cpu = cpu_baseline(args.cpu_seconds)
         extras = None
         if world == 1 and not args.no_extras:
-            extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement()}
+            extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement(),
+                      "multi_query_32x4096": multi_query_measurement()}
         steps_per_s = args.steps / (ms_max / 1000) * world
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

@@ -533,7 +533,9 @@ int run_decode(const Geometry& geo, const DecodeArgs& args, const void* k, const
                cudaStream_t stream) {
   auto per_g = [&](auto gc) -> int {
     constexpr int G = decltype(gc)::value;
-    if constexpr (sizeof(T) == 2 && G <= 8) {
+    // tensor-core tiles for bf16: up to 16 columns at head_dim <= 128 (two
+    // 8-column blocks), up to 8 at head_dim 256 (their registers run out)
+    if constexpr (sizeof(T) == 2 && (G <= 8 || D <= 128)) {
       if (args.block_size >= 8 && g_kernel_choice != 1)
         return launch_core<MmaCore<D, G>, G>(geo, args, k, v, stream);
     }

@@ -82,7 +82,8 @@ def test_tiny_nine_requests_in_one_pool_fail_cleanly():
 
 
 @pytest.mark.parametrize("B", [4, 8, 16, 32, 64])
-@pytest.mark.parametrize("G,Hkv,D", [(4, 8, 128), (8, 4, 128), (1, 4, 64), (2, 2, 64), (4, 2, 256)])
+@pytest.mark.parametrize("G,Hkv,D", [(4, 8, 128), (8, 4, 128), (1, 4, 64), (2, 2, 64), (4, 2, 256),
+                                     (16, 2, 128), (16, 1, 64)])
 def test_bf16_mixed_lengths(kernel, B, G, Hkv, D):
     import torch
 
