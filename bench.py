@@ -17,6 +17,8 @@ Reported (one JSON line from rank 0):
                K/V written + block tables and lengths
   e2e          the same metric with q, new K/V from pinned host buffers and
                the outputs read back to the host inside the timed region
+               (per-layer copies on two copy streams, overlapped with the
+               other layers' attention)
   roofline     paged decode attention (one partition-kernel launch per layer,
                append and merge folded in): bytes per launch / average launch
                duration, from CUDA events around each step's layer loop in the
@@ -227,9 +229,13 @@ class DecodeStep:
         for _ in range(L):
             self.k_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
             self.v_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
-        self.q = [torch.randn((S, Hq, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
-        self.k_new = [torch.randn((S, Hkv, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
-        self.v_new = [torch.randn((S, Hkv, D), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        # per layer one packed input row [q | k_new | v_new], so the end-to-end
+        # pass moves each layer's inputs with one host->device copy
+        nq, nkv = S * Hq * D, S * Hkv * D
+        self.in_d = torch.randn((L, nq + 2 * nkv), generator=gen, device=dev, dtype=torch.bfloat16)
+        self.q = [self.in_d[i, :nq].view(S, Hq, D) for i in range(L)]
+        self.k_new = [self.in_d[i, nq:nq + nkv].view(S, Hkv, D) for i in range(L)]
+        self.v_new = [self.in_d[i, nq + nkv:].view(S, Hkv, D) for i in range(L)]
         self.out = [torch.empty((S, Hq, D), device=dev, dtype=torch.bfloat16) for _ in range(L)]
         self.status = np.zeros(S, dtype=np.int32)
         self.copies_h = np.zeros((S, 3), dtype=np.int32)
@@ -252,11 +258,15 @@ class DecodeStep:
         self.attn_bytes = []
         self.attn_events = []
         self.record_attn = False
-        # e2e host buffers
-        self.q_h = [self.q[i].cpu().pin_memory() for i in range(L)]
-        self.kn_h = [self.k_new[i].cpu().pin_memory() for i in range(L)]
-        self.vn_h = [self.v_new[i].cpu().pin_memory() for i in range(L)]
+        # e2e host buffers and copy streams: layer l's inputs go up on one stream
+        # while earlier layers compute, its output comes back on another
+        self.in_h = self.in_d.cpu().pin_memory()
         self.out_h = [torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+        self.up = torch.cuda.Stream()
+        self.down = torch.cuda.Stream()
+        self.in_ready = [torch.cuda.Event() for _ in range(L)]   # layer inputs on the device
+        self.used = [None] * L                                  # layer inputs consumed (last step)
+        self.out_read = [None] * L                              # layer output read back (last step)
 
     def bytes_of_step(self, lens: np.ndarray, n_copies: int) -> int:
         """Algorithmic bytes: every history slot read once per KV head, q, out, appends, metadata."""
@@ -307,13 +317,20 @@ class DecodeStep:
         self.launches += 2
         if e2e:
             for i in range(self.L):
-                self.q[i].copy_(self.q_h[i], non_blocking=True)
-                self.k_new[i].copy_(self.kn_h[i], non_blocking=True)
-                self.v_new[i].copy_(self.vn_h[i], non_blocking=True)
+                # one copy per layer, after the previous step's layer i has consumed its inputs
+                if self.used[i] is not None:
+                    self.up.wait_event(self.used[i])
+                with torch.cuda.stream(self.up):
+                    self.in_d[i].copy_(self.in_h[i], non_blocking=True)
+                self.in_ready[i].record(self.up)
         if self.record_attn:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(self.stream)
         for i in range(self.L):
+            if e2e:
+                self.stream.wait_event(self.in_ready[i])
+                if self.out_read[i] is not None:   # the previous step's output i has left the device
+                    self.stream.wait_event(self.out_read[i])
             if not self.fused:
                 pkv.kv_append(self.k_new[i], self.v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
                 self.launches += 1
@@ -325,13 +342,23 @@ class DecodeStep:
                 pkv.paged_decode_attn_run(self.q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
                                           self.wl.scale, self.out[i], self.ws)
             self.launches += 1
+            if e2e:
+                done = torch.cuda.Event()
+                done.record(self.stream)
+                self.used[i] = done
+                self.down.wait_event(done)
+                with torch.cuda.stream(self.down):
+                    self.out_h[i].copy_(self.out[i], non_blocking=True)
+                back = torch.cuda.Event()
+                back.record(self.down)
+                self.out_read[i] = back
         if self.record_attn:
             e1.record(self.stream)
             self.attn_events.append((e0, e1))
             self.attn_bytes.append(self.attn_bytes_per_launch(lens))
         if e2e:
-            for i in range(self.L):
-                self.out_h[i].copy_(self.out[i], non_blocking=True)
+            # the step ends when its last output is on the host
+            self.stream.wait_event(self.out_read[self.L - 1])
         self.bytes_done += self.bytes_of_step(lens, nc)
 
     def h2d_d2h_bytes(self):
