@@ -63,7 +63,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
-    p.add_argument("--no-extras", action="store_true", help="skip the swap and allocator measurements")
+    p.add_argument("--no-extras", action="store_true", help="skip the measurements of the other rows")
+    p.add_argument("--extra", default=None,
+                   choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving"],
+                   help="run only this one extra measurement and print its JSON (for profiling captures)")
     p.add_argument("--unfused", action="store_true",
                    help="append with a separate kv_append launch instead of folding it into attention")
     p.add_argument("--layers", type=int, default=32,
@@ -509,6 +512,100 @@ def multi_query_measurement(reps: int = 20):
     return res
 
 
+def _time_decode(pkv, torch, q, pools, tables, lens, scale, ws, reps):
+    """Average microseconds of one paged_decode_attn call (plan + attention),
+    rotating over the pool copies so every call streams from HBM."""
+    for i in range(2):
+        pkv.paged_decode_attn(q, pools[i][0], pools[i][1], tables, lens, scale, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        kp, vp = pools[i % len(pools)]
+        pkv.paged_decode_attn(q, kp, vp, tables, lens, scale, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000 / reps
+
+
+def prefix_cow_measurement(reps: int = 20):
+    """Shared prompts: 64 groups x 4 branches fork one 2008-token prompt (full
+    blocks shared, the 8-token tail copied on the first append) and append 256
+    tokens each; one layer (H_q 16, H_kv 4, d 128, bf16, B 16).  Reports the
+    logical KV GB/s (every request's whole history counted) and the unique
+    GB/s (each physical block counted once): shared blocks may be served from
+    L2 for the later branches of a group."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    import workloads as W
+
+    wl = W.workload("prefix_cow")
+    G, BR, P, A = 64, 4, 2008, 256
+    S, Hq, Hkv, D, B, N = G * BR, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.pool_blocks
+    a = pkv.BlockAllocator(N, B, free_order=W.free_order(W.rng(wl.seed), N))
+    ids = []
+    for g in range(G):
+        root = g * BR
+        assert a.add_seq(root, P) == 0
+        for b in range(1, BR):
+            assert a.fork(root, root + b) == 0
+        ids += list(range(root, root + BR))
+    ids = np.array(ids, dtype=np.int32)
+    st = np.zeros(S, dtype=np.int32)
+    cp = np.zeros((S, 3), dtype=np.int32)
+    copies = 0
+    for _ in range(A):
+        rc, nc = a.append_arrays(ids, st, cp)
+        assert rc == 0
+        copies += nc
+    tables, lens = a.fill_tables(list(ids), -(-(P + A) // B))
+    unique_blocks = a.stats()["active"]
+    td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    pools = [(torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16),
+              torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16)) for _ in range(8)]
+    q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
+    ws = pkv.new_workspace(S, Hq, Hkv, D)
+    us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
+    row = Hkv * D * 2 * 2
+    logical = int(lens.sum()) * row + 2 * S * Hq * D * 2
+    unique = unique_blocks * B * row + 2 * S * Hq * D * 2
+    del pools
+    return {"us_per_layer": us, "logical_gb_per_s": logical / (us * 1e-6) / 1e9,
+            "unique_gb_per_s": unique / (us * 1e-6) / 1e9, "cow_copies": copies,
+            "logical_mb": logical / 1e6, "unique_mb": unique / 1e6}
+
+
+def large_serving_measurement(reps: int = 12):
+    """256 requests with lengths uniform in 1..8192, H_q 32, H_kv 4 (G = 8),
+    d 128, bf16, B 16, shuffled tables; one layer per call."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    import workloads as W
+
+    wl = W.workload("large_serving")
+    S, Hq, Hkv, D, B, N = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.pool_blocks
+    a = pkv.BlockAllocator(N, B, free_order=W.free_order(W.rng(wl.seed), N))
+    for i, n in enumerate(wl.lengths):
+        assert a.add_seq(i, n) == 0
+    tables, lens = a.fill_tables(list(range(S)), -(-max(wl.lengths) // B))
+    td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9)
+    pools = [(torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16),
+              torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16)) for _ in range(3)]
+    q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
+    ws = pkv.new_workspace(S, Hq, Hkv, D)
+    us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
+    nbytes = (int(lens.sum()) * Hkv * D * 2 * 2 + 2 * S * Hq * D * 2
+              + 4 * int(sum(-(-int(n) // B) for n in lens)) + 4 * S)
+    del pools
+    return {"us_per_layer": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9, "kv_tokens": int(lens.sum())}
+
+
 def allocator_measurement(seconds: float = 1.0):
     """Host allocator throughput (C++): admit with prefix-cache hits, decode
     appends, release, on a 4096-block pool; operations per second."""
@@ -584,10 +681,22 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+EXTRAS = {
+    "swap": lambda: swap_measurement(),
+    "allocator": lambda: allocator_measurement(),
+    "multi_query": lambda: multi_query_measurement(),
+    "prefix_cow": lambda: prefix_cow_measurement(),
+    "large_serving": lambda: large_serving_measurement(),
+}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.extra is not None:
+        print(json.dumps({args.extra: EXTRAS[args.extra]()}), flush=True)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
     import torch
@@ -647,7 +756,9 @@ def main():
         extras = None
         if world == 1 and not args.no_extras:
             extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement(),
-                      "multi_query_32x4096": multi_query_measurement()}
+                      "multi_query_32x4096": multi_query_measurement(),
+                      "prefix_cow_256x2264": prefix_cow_measurement(),
+                      "large_serving_256xU8192": large_serving_measurement()}
         steps_per_s = args.steps / (ms_max / 1000) * world
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
