@@ -67,6 +67,8 @@ def parse():
     p.add_argument("--extra", default=None,
                    choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving"],
                    help="run only this one extra measurement and print its JSON (for profiling captures)")
+    p.add_argument("--no-overlap", action="store_true",
+                   help="launch every layer's attention without programmatic dependent launch")
     p.add_argument("--unfused", action="store_true",
                    help="append with a separate kv_append launch instead of folding it into attention")
     p.add_argument("--layers", type=int, default=32,
@@ -202,7 +204,7 @@ class DecodeStep:
     """32-layer decode step through the C ABI; all state resident on the device."""
 
     def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1,
-                 layers: int = 32, fused: bool = True):
+                 layers: int = 32, fused: bool = True, overlap: bool = True):
         import torch
 
         import paged_kv_cache_358_b200 as pkv
@@ -210,6 +212,10 @@ class DecodeStep:
 
         self.torch, self.pkv = torch, pkv
         self.fused = fused
+        # layers after the first may start while the previous layer's launch
+        # finishes (each reads its own pool; the plan, tables and slots were
+        # written by kernels that completed before layer 0 started)
+        self.overlap = overlap
         pkv.set_decode_kernel(kernel)
         wl = W.workload("teaching_32x4096", decode_steps=steps_budget + 8, seed=seed)
         self.wl = wl
@@ -232,14 +238,17 @@ class DecodeStep:
         for _ in range(L):
             self.k_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
             self.v_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
-        # per layer one packed input row [q | k_new | v_new], so the end-to-end
-        # pass moves each layer's inputs with one host->device copy
+        # a step's inputs, per layer one packed row [q | k_new | v_new], and its
+        # outputs are each one contiguous buffer, two of each: the end-to-end
+        # pass moves a step's inputs with one host->device copy and its outputs
+        # with one device->host copy, while the neighbouring step computes
         nq, nkv = S * Hq * D, S * Hkv * D
-        self.in_d = torch.randn((L, nq + 2 * nkv), generator=gen, device=dev, dtype=torch.bfloat16)
-        self.q = [self.in_d[i, :nq].view(S, Hq, D) for i in range(L)]
-        self.k_new = [self.in_d[i, nq:nq + nkv].view(S, Hkv, D) for i in range(L)]
-        self.v_new = [self.in_d[i, nq + nkv:].view(S, Hkv, D) for i in range(L)]
-        self.out = [torch.empty((S, Hq, D), device=dev, dtype=torch.bfloat16) for _ in range(L)]
+        self.in_d = torch.randn((2, L, nq + 2 * nkv), generator=gen, device=dev, dtype=torch.bfloat16)
+        self.q = [[self.in_d[b, i, :nq].view(S, Hq, D) for i in range(L)] for b in range(2)]
+        self.k_new = [[self.in_d[b, i, nq:nq + nkv].view(S, Hkv, D) for i in range(L)] for b in range(2)]
+        self.v_new = [[self.in_d[b, i, nq + nkv:].view(S, Hkv, D) for i in range(L)] for b in range(2)]
+        self.out_d = torch.empty((2, L, S, Hq, D), device=dev, dtype=torch.bfloat16)
+        self.out = [[self.out_d[b, i] for i in range(L)] for b in range(2)]
         self.status = np.zeros(S, dtype=np.int32)
         self.copies_h = np.zeros((S, 3), dtype=np.int32)
         # pinned double buffers for the tables and lengths mirrored each step
@@ -261,15 +270,17 @@ class DecodeStep:
         self.attn_bytes = []
         self.attn_events = []
         self.record_attn = False
-        # e2e host buffers and copy streams: layer l's inputs go up on one stream
-        # while earlier layers compute, its output comes back on another
-        self.in_h = self.in_d.cpu().pin_memory()
-        self.out_h = [torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+        # e2e host buffers and copy streams: step k's inputs go up on one stream
+        # (while step k-1 computes) and its outputs come back on another (while
+        # step k+1 computes); events order every copy against the kernels
+        self.in_h = self.in_d[0].cpu().pin_memory()
+        self.out_h = torch.empty((2, L, S, Hq, D), dtype=torch.bfloat16).pin_memory()
         self.up = torch.cuda.Stream()
         self.down = torch.cuda.Stream()
-        self.in_ready = [torch.cuda.Event() for _ in range(L)]   # layer inputs on the device
-        self.used = [None] * L                                  # layer inputs consumed (last step)
-        self.out_read = [None] * L                              # layer output read back (last step)
+        self.e2e_k = 0
+        self.in_ready = [None, None]    # per buffer: inputs of its current step on the device
+        self.step_done = [None, None]   # per buffer: its step's kernels finished
+        self.out_back = [None, None]    # per buffer: its step's outputs on the host
 
     def bytes_of_step(self, lens: np.ndarray, n_copies: int) -> int:
         """Algorithmic bytes: every history slot read once per KV head, q, out, appends, metadata."""
@@ -318,51 +329,58 @@ class DecodeStep:
         pkv.slot_mapping(self.tab_d, self.pos_d, self.B, out=self.slots)
         pkv.decode_plan(self.len_d, self.Hq, self.Hkv, self.D, pkv.BF16, self.ws)
         self.launches += 2
+        eb = 0
         if e2e:
-            for i in range(self.L):
-                # one copy per layer, after the previous step's layer i has consumed its inputs
-                if self.used[i] is not None:
-                    self.up.wait_event(self.used[i])
-                with torch.cuda.stream(self.up):
-                    self.in_d[i].copy_(self.in_h[i], non_blocking=True)
-                self.in_ready[i].record(self.up)
+            eb = self.e2e_k % 2
+            self.e2e_k += 1
+            # upload this step's inputs once the step that last used the buffer is done
+            if self.step_done[eb] is not None:
+                self.up.wait_event(self.step_done[eb])
+            with torch.cuda.stream(self.up):
+                self.in_d[eb].copy_(self.in_h, non_blocking=True)
+            self.in_ready[eb] = torch.cuda.Event()
+            self.in_ready[eb].record(self.up)
+            self.stream.wait_event(self.in_ready[eb])
+            if self.out_back[eb] is not None:   # the outputs last written here are on the host
+                self.stream.wait_event(self.out_back[eb])
         if self.record_attn:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(self.stream)
+        q, k_new, v_new, out = self.q[eb], self.k_new[eb], self.v_new[eb], self.out[eb]
         for i in range(self.L):
-            if e2e:
-                self.stream.wait_event(self.in_ready[i])
-                if self.out_read[i] is not None:   # the previous step's output i has left the device
-                    self.stream.wait_event(self.out_read[i])
             if not self.fused:
-                pkv.kv_append(self.k_new[i], self.v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
+                pkv.kv_append(k_new[i], v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
                 self.launches += 1
+            pkv.set_launch_overlap(self.overlap and i > 0 and self.fused)
             if self.fused:
-                pkv.paged_decode_attn_append_run(self.q[i], self.k_new[i], self.v_new[i], self.slots,
+                pkv.paged_decode_attn_append_run(q[i], k_new[i], v_new[i], self.slots,
                                                  self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
-                                                 self.wl.scale, self.out[i], self.ws)
+                                                 self.wl.scale, out[i], self.ws)
             else:
-                pkv.paged_decode_attn_run(self.q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
-                                          self.wl.scale, self.out[i], self.ws)
+                pkv.paged_decode_attn_run(q[i], self.k_pools[i], self.v_pools[i], self.tab_d, self.len_d,
+                                          self.wl.scale, out[i], self.ws)
             self.launches += 1
-            if e2e:
-                done = torch.cuda.Event()
-                done.record(self.stream)
-                self.used[i] = done
-                self.down.wait_event(done)
-                with torch.cuda.stream(self.down):
-                    self.out_h[i].copy_(self.out[i], non_blocking=True)
-                back = torch.cuda.Event()
-                back.record(self.down)
-                self.out_read[i] = back
+        pkv.set_launch_overlap(False)
+        if e2e:
+            done = torch.cuda.Event()
+            done.record(self.stream)
+            self.step_done[eb] = done
+            self.down.wait_event(done)
+            with torch.cuda.stream(self.down):
+                self.out_h[eb].copy_(self.out_d[eb], non_blocking=True)
+            self.out_back[eb] = torch.cuda.Event()
+            self.out_back[eb].record(self.down)
         if self.record_attn:
             e1.record(self.stream)
             self.attn_events.append((e0, e1))
             self.attn_bytes.append(self.attn_bytes_per_launch(lens))
-        if e2e:
-            # the step ends when its last output is on the host
-            self.stream.wait_event(self.out_read[self.L - 1])
         self.bytes_done += self.bytes_of_step(lens, nc)
+
+    def drain(self):
+        """Order the compute stream after the last outputs' copy to the host."""
+        for ev in self.out_back:
+            if ev is not None:
+                self.stream.wait_event(ev)
 
     def h2d_d2h_bytes(self):
         e = 2
@@ -371,7 +389,7 @@ class DecodeStep:
         return self.L * per_layer_in + meta, self.L * self.S * self.Hq * self.D * e
 
 
-def timed(fn, steps, dist, stream):
+def timed(fn, steps, dist, stream, finish=None):
     import torch
 
     if dist is not None:
@@ -382,6 +400,8 @@ def timed(fn, steps, dist, stream):
     e0.record(stream)
     for _ in range(steps):
         fn()
+    if finish is not None:
+        finish()
     e1.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - w0
@@ -704,7 +724,8 @@ def main():
     rank, world, dist = dist_init(args.gpus)
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     budget = 2 * (args.warmup + args.steps) + 6
-    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world, args.layers, not args.unfused)
+    ds = DecodeStep(budget, args.seed + rank, args.kernel, rank, world, args.layers, not args.unfused,
+                    not args.no_overlap)
     stream = ds.stream
     for _ in range(args.warmup):
         ds.step()
@@ -734,7 +755,7 @@ def main():
     for _ in range(2):
         ds.step(e2e=True)
     ds.bytes_done = 0
-    ms_e2e, _ = timed(lambda: ds.step(e2e=True), args.steps, dist, stream)
+    ms_e2e, _ = timed(lambda: ds.step(e2e=True), args.steps, dist, stream, finish=ds.drain)
     e2e_bytes = ds.bytes_done
     h2d, d2h = ds.h2d_d2h_bytes()
 
@@ -769,7 +790,8 @@ def main():
                        "H_q": ds.Hq, "H_kv": ds.Hkv, "head_dim": ds.D, "block_size": ds.B,
                        "pool_blocks_per_layer": ds.N, "kv_pool_gib": round(2 * ds.L * ds.N * ds.B * ds.Hkv * ds.D * 2 / 2**30, 2),
                        "l2": "inputs larger than L2 (KV pool far above 126 MB); no flush",
-                       "parallelism": f"replicas x{world} (requests sharded by rank, no collective)"},
+                       "parallelism": f"replicas x{world} (requests sharded by rank, no collective)",
+                       "launch_overlap": bool(ds.overlap and ds.fused)},
             "steps_per_s": steps_per_s, "tokens_per_s": steps_per_s * ds.S,
             "frac_of_nominal_8tbs": value / NOMINAL_HBM_GBS,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -777,7 +799,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": ("paged_decode_attn_append_run (append and merge folded in)" if ds.fused else
-                                    "paged_decode_attn_run (merge folded in)") + ", 32x4096, one layer per launch",
+                                    "paged_decode_attn_run (merge folded in)") + ", 32x4096, one layer per launch"
+                                   + ("; layers 2..32 overlap their predecessor's tail (programmatic dependent "
+                                      "launch), so the per-launch time is the layer loop's span / 32"
+                                      if ds.overlap and ds.fused else ""),
                          "avg_launch_us": avg_attn_ms * 1000,
                          "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu,

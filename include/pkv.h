@@ -238,6 +238,21 @@ int pkv_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size
  * storage always uses FMA tiles.  Process-wide; for measurement. */
 int pkv_set_decode_kernel(int32_t which);
 
+/* Launch overlap (default 0 = off).  With 1, pkv_paged_decode_attn_run and
+ * pkv_paged_decode_attn_append_run launch as programmatic dependent launches:
+ * their CTAs may start while the kernel launched just before them on the
+ * stream is still finishing, read the plan, block tables, lengths, slot
+ * mapping and this call's K/V pool, and start their first K/V loads; they
+ * wait for that kernel to complete (and its writes to be visible) before
+ * reading q, k_new or v_new and before writing anything.  Set it only for
+ * calls where the kernel launched immediately before does not write the
+ * workspace plan, the block tables, seq_lens, the slot mapping or the K/V
+ * pool the call reads: e.g. layers 2..L of one decode step, each reading its
+ * own pool, but not the first layer right after pkv_decode_plan.  The calls
+ * that plan themselves (pkv_paged_decode_attn, pkv_paged_attn_multi_query,
+ * the allocation-free call) never overlap.  Process-wide; read at launch. */
+int pkv_set_launch_overlap(int32_t on);
+
 /* ==========================================================================
  * Cache writes
  * ==========================================================================

@@ -18,7 +18,8 @@ __all__ = [
     "lib", "library_path", "Status", "PkvError",
     "BF16", "F32",
     "decode_workspace_bytes", "paged_decode_attn", "decode_plan", "paged_decode_attn_run",
-    "decode_status", "set_decode_kernel", "paged_decode_attn_append_run", "paged_attn_multi_query",
+    "decode_status", "set_decode_kernel", "set_launch_overlap", "paged_decode_attn_append_run",
+    "paged_attn_multi_query",
     "kv_append", "block_copy", "slot_mapping", "swap_blocks",
     "BlockAllocator",
 ]
@@ -83,6 +84,7 @@ _SIGS = {
     "pkv_paged_attn_multi_query": (ctypes.c_int, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                   _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
+    "pkv_set_launch_overlap": (ctypes.c_int, [_i32]),
     "pkv_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_ulonglong, _vp, _sz, _vp]),
     "pkv_kv_append": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_block_copy": (ctypes.c_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _vp, _i32, _i32, _i32,
@@ -282,6 +284,11 @@ def decode_status(workspace, stream=None) -> int:
 def set_decode_kernel(which: int) -> None:
     """0 automatic, 1 CUDA-core FMA tiles, 2 tensor-core tiles (bf16)."""
     _check(lib().pkv_set_decode_kernel(int(which)), "set_decode_kernel")
+
+
+def set_launch_overlap(on: bool) -> None:
+    """Programmatic dependent launch of the decode kernels (see pkv_set_launch_overlap)."""
+    _check(lib().pkv_set_launch_overlap(1 if on else 0), "set_launch_overlap")
 
 
 def kv_append(k, v, slot_mapping, k_pool, v_pool, stream=None) -> None:

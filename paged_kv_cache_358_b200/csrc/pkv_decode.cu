@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 namespace pkv {
 
 int g_kernel_choice = 0;
+int g_launch_overlap = 0;
 
 namespace {
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -295,7 +296,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
-             int32_t num_q_tokens = 1) {
+             int32_t num_q_tokens = 1, bool overlap = false) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -334,6 +335,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.out_dtype = out_dtype;
   args.num_workers = geo.NW;
   args.num_q_tokens = num_q_tokens;
+  geo.overlap = overlap;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
   args.v_new = new_slots ? v_new : nullptr;
@@ -367,7 +369,7 @@ int pkv_paged_decode_attn_run(const void* q, const void* k_pool, const void* v_p
                               pkv_stream_t stream) {
   return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                   num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
-                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr);
+                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, 1, g_launch_overlap != 0);
 }
 
 int pkv_paged_decode_attn_append_run(const void* q, const void* k_new, const void* v_new,
@@ -381,7 +383,7 @@ int pkv_paged_decode_attn_append_run(const void* q, const void* k_new, const voi
   if (num_seqs > 0 && !slot_mapping) return PKV_ERR_INVALID;
   return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                   num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
-                  workspace, workspace_bytes, stream, k_new, v_new, slot_mapping);
+                  workspace, workspace_bytes, stream, k_new, v_new, slot_mapping, 1, g_launch_overlap != 0);
 }
 
 int pkv_paged_decode_attn(const void* q, const void* k_pool, const void* v_pool,
@@ -400,10 +402,10 @@ int pkv_paged_decode_attn(const void* q, const void* k_pool, const void* v_pool,
   if (num_seqs == 0) return PKV_OK;
   rc = do_plan(geo, seq_lens, workspace, static_cast<cudaStream_t>(stream));
   if (rc != PKV_OK) return rc;
-  return pkv_paged_decode_attn_run(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens,
-                                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                   num_blocks, scale, kv_dtype, out, out_dtype, workspace,
-                                   workspace_bytes, stream);
+  // the plan kernel just launched writes what the attention reads first: no overlap
+  return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                  num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
+                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, 1, false);
 }
 
 int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* k_pool, const void* v_pool,
@@ -481,6 +483,12 @@ int pkv_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size
 int pkv_set_decode_kernel(int32_t which) {
   if (which < 0 || which > 2) return PKV_ERR_INVALID;
   g_kernel_choice = which;
+  return PKV_OK;
+}
+
+int pkv_set_launch_overlap(int32_t on) {
+  if (on != 0 && on != 1) return PKV_ERR_INVALID;
+  g_launch_overlap = on;
   return PKV_OK;
 }
 

@@ -174,19 +174,27 @@ __global__ void __launch_bounds__(W * 32, CPS)
   int32_t* bt = reinterpret_cast<int32_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta + SM::kBatchB);
 
+  // The next kernel of the stream may be scheduled now; it starts on an SM
+  // as this launch's CTAs leave it.
+  if (threadIdx.x == 0) grid_launch_dependents();
+  // Until grid_dependency_wait() below, this launch only reads what the
+  // kernel just before it does not write (plan, tables, lengths, slots, K/V
+  // pool), through L2, and writes no global memory but error flags.
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
   uint32_t* status = &hdr->status;
-  if (hdr->planned != 1 || hdr->num_seqs != check_S || hdr->num_q_heads != check_Hq ||
-      hdr->num_kv_heads != check_Hkv || hdr->head_dim != check_D || hdr->kv_dtype != check_dtype ||
-      hdr->num_workers != a.num_workers || hdr->head_groups != a.head_groups) {
+  if (__ldcg(&hdr->planned) != 1 || __ldcg(&hdr->num_seqs) != check_S || __ldcg(&hdr->num_q_heads) != check_Hq ||
+      __ldcg(&hdr->num_kv_heads) != check_Hkv || __ldcg(&hdr->head_dim) != check_D ||
+      __ldcg(&hdr->kv_dtype) != check_dtype || __ldcg(&hdr->num_workers) != a.num_workers ||
+      __ldcg(&hdr->head_groups) != a.head_groups) {
+    grid_dependency_wait();
     if (threadIdx.x == 0) record_status(status, kStatusPlanMismatch);
     return;
   }
-  const long long TT = hdr->total_tiles;
+  const long long TT = __ldcg(&hdr->total_tiles);
   const int NW = a.num_workers;
   const int v = blockIdx.x;  // this CTA's worker id; warp = head within the group
-  const int4 wp = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[2 * v];
-  const int first_len = reinterpret_cast<const int4*>(a.ws + a.off_wplan)[2 * v + 1].x;
+  const int4 wp = __ldcg(reinterpret_cast<const int4*>(a.ws + a.off_wplan) + 2 * v);
+  const int first_len = __ldcg(reinterpret_cast<const int4*>(a.ws + a.off_wplan) + 2 * v + 1).x;
   const int ntiles = wp.y - wp.x;
 
   const int S = a.num_seqs, Hkv = a.num_kv_heads, NHG = a.head_groups, Bsz = a.block_size;
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
           break;
         }
         ++s;
-        len = a.seq_lens[s];
+        len = __ldcg(a.seq_lens + s);
         nt = ntiles_of(len);
       }
       const int hg = nt > 0 ? off / nt : 0;
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       n_nt = nt;
       n_flags = (min(kTile, len - j * kTile) << 8) | (j == nt - 1 ? 2 : 0);
       n_len = len;
-      n_slot = (a.new_slots != nullptr && j == nt - 1) ? a.new_slots[s] : -1;
+      n_slot = (a.new_slots != nullptr && j == nt - 1) ? __ldcg(a.new_slots + s) : -1;
       const int32_t* row = a.block_tables + static_cast<size_t>(s) * a.max_blocks;
 #pragma unroll
       for (int b = 0; b < kMaxBoxes; ++b) {
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
           if (lb0 + b >= a.max_blocks) {
             n_over |= 1u << b;
           } else {
-            n_phys[b] = row[lb0 + b];
+            n_phys[b] = __ldcg(row + lb0 + b);
             n_have |= 1u << b;
           }
         }
@@ -313,6 +321,20 @@ __global__ void __launch_bounds__(W * 32, CPS)
   };
 
   int last_s = -1, last_hg = -1;
+  // q is written by earlier kernels: in the prologue (before the dependency
+  // wait) a stage's q copy is held back, and the stage's arrival with it.
+  bool defer_q = true;
+  uint32_t q_pending = 0;  // lane 0: stages whose q copy and arrival wait
+  auto load_q = [&](int st, int s, int head) {
+    char* stage = stages + st * Core::kStageBytes;
+    const uint32_t bar = smem_u32(&bars[st]);
+    // the pair's G columns: Gq grouped heads of each of the T query tokens
+    for (int i = 0; i < T; ++i) {
+      const char* qsrc = reinterpret_cast<const char*>(a.q) +
+                         ((static_cast<size_t>(s) * T + i) * Hq + static_cast<size_t>(head) * Gq) * Core::ROWB;
+      bulk_load(smem_u32(stage + Core::kQOff + i * Gq * Core::ROWB), qsrc, Gq * Core::ROWB, bar);
+    }
+  };
   auto issue = [&](int k) {
     if ((k % kBatch) == 0) {
       commit();               // batch k, loaded during the previous batch
@@ -342,14 +364,12 @@ __global__ void __launch_bounds__(W * 32, CPS)
       uint32_t bytes = 2u * nb * Core::kChunks * box_bytes;
       if (newpair) bytes += ncols * Core::ROWB;
       fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, bytes);
-      if (newpair) {
-        // the pair's G columns: Gq grouped heads of each of the T query tokens
-        for (int i = 0; i < T; ++i) {
-          const char* qsrc = reinterpret_cast<const char*>(a.q) +
-                             ((static_cast<size_t>(s) * T + i) * Hq + static_cast<size_t>(head) * Gq) * Core::ROWB;
-          bulk_load(smem_u32(stage + Core::kQOff + i * Gq * Core::ROWB), qsrc, Gq * Core::ROWB, bar);
-        }
+      if (newpair && defer_q) {
+        mbar_expect_tx(bar, bytes);  // arrival after the q copy, past the dependency wait
+        q_pending |= 1u << st;
+      } else {
+        mbar_arrive_expect_tx(bar, bytes);
+        if (newpair) load_q(st, s, head);
       }
       const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
 #pragma unroll
@@ -375,6 +395,19 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const int prologue = ntiles < DEPTH ? ntiles : DEPTH;
     for (int k = 0; k < prologue; ++k) issue(k);
   }
+  // Everything below may read what earlier kernels wrote (q, k_new, v_new)
+  // and writes global memory.
+  grid_dependency_wait();
+  defer_q = false;
+  if (lane == 0) {
+    for (int st = 0; st < DEPTH; ++st) {
+      if (q_pending & (1u << st)) {
+        load_q(st, meta[st].s, meta[st].hg * W + warp);
+        mbar_arrive(smem_u32(&bars[st]));
+      }
+    }
+  }
+  __syncwarp();
 
   // Requests of length 0 produce zeros; CTA v writes those of pairs v, v + NW, ...
   for (long long p = v; p < static_cast<long long>(S) * NHG; p += NW) {
@@ -482,6 +515,7 @@ struct Geometry {
   int S, Hq, Hkv, G, D, dtype;
   int HG, NHG, CPS, NW;
   WsLayout lay;
+  bool overlap = false;  // launch as a programmatic dependent launch
 };
 
 extern int g_kernel_choice;  // 0 auto, 1 CUDA-core tiles, 2 tensor-core tiles (bf16)
@@ -513,7 +547,22 @@ int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_
     if (e != cudaSuccess) return host::cuda_fail(e);
     configured_dev = dev;
   }
-  kern<<<geo.NW, W * 32, SM::kTotal, stream>>>(maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
+  if (!geo.overlap) {
+    kern<<<geo.NW, W * 32, SM::kTotal, stream>>>(maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
+    return host::check_launch();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(geo.NW);
+  cfg.blockDim = dim3(W * 32);
+  cfg.dynamicSmemBytes = SM::kTotal;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
+  if (e != cudaSuccess) return host::cuda_fail(e);
   return host::check_launch();
 }
 
