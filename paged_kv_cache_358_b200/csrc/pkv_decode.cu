@@ -1,9 +1,10 @@
 // Decode attention entry points of libpkv: the plan kernel, the host side that
 // validates arguments and builds the TMA tensor maps, and the C ABI.  The
-// partition kernel (persistent stream-K over CTAs; the warps of a CTA take the
-// KV heads of one head group over the same 16-token tiles; the last CTA on a
-// split request merges the partial states) lives in pkv_decode_kernels.cuh and
-// is instantiated per (storage type, head_dim) in pkv_decode_<type>_<d>.cu.
+// partition kernel (persistent stream-K over one-warp CTAs, each taking an
+// equal range of (request, KV head, 16-token tile) units; the last CTA on a
+// split (request, KV head) merges the partial states) lives in
+// pkv_decode_kernels.cuh and is instantiated per (storage type, head_dim) in
+// pkv_decode_<type>_<d>.cu.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
