@@ -221,7 +221,6 @@ def test_swap_500mib_time_against_the_pages_estimate():
     """Move 500 MiB of KV out and back and report the time next to the pages' analytic
     19.5 ms one way at 25 GiB/s (the measured link may be faster or slower)."""
     import json
-    import os
 
     import torch
 
@@ -248,7 +247,5 @@ def test_swap_500mib_time_against_the_pages_estimate():
     rec = {"mib": 500, "out_ms": times["out"], "in_ms": times["in"],
            "out_gib_per_s": 500 / 1024 / (times["out"] / 1000), "in_gib_per_s": 500 / 1024 / (times["in"] / 1000),
            "pages_one_way_ms_at_25_gib_per_s": 19.5}
-    os.makedirs("gpurun_out", exist_ok=True)
-    with open("gpurun_out/swap_500mib.json", "w") as f:
-        json.dump(rec, f)
+    print("swap 500 MiB:", json.dumps(rec))
     assert times["out"] > 0 and times["in"] > 0
