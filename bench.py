@@ -589,13 +589,38 @@ def prefix_cow_measurement(reps: int = 20):
     q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
     ws = pkv.new_workspace(S, Hq, Hkv, D)
     us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
+    # the same batch through the shared-prefix call: each group's 125 full
+    # prompt blocks are read once for its 4 branches
+    gs = torch.arange(0, S + 1, BR, dtype=torch.int32, device="cuda")
+    pb = torch.full((G,), P // B, dtype=torch.int32, device="cuda")
+    wsp = pkv.shared_prefix_workspace(S, G, BR, Hq, Hkv, D, tables.shape[1])
+    out = torch.empty((S, Hq, D), dtype=torch.bfloat16, device="cuda")
+
+    def shared(i):
+        kp, vp = pools[i % len(pools)]
+        pkv.paged_decode_attn_shared_prefix(q, kp, vp, td, ld, gs, pb, BR, wl.scale, out=out, workspace=wsp)
+
+    for i in range(2):
+        shared(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        shared(i)
+    e1.record()
+    torch.cuda.synchronize()
+    us_shared = e0.elapsed_time(e1) * 1000 / reps
+    assert pkv.decode_status(wsp) == 0
     row = Hkv * D * 2 * 2
     logical = int(lens.sum()) * row + 2 * S * Hq * D * 2
     unique = unique_blocks * B * row + 2 * S * Hq * D * 2
     del pools
     return {"us_per_layer": us, "logical_gb_per_s": logical / (us * 1e-6) / 1e9,
             "unique_gb_per_s": unique / (us * 1e-6) / 1e9, "cow_copies": copies,
-            "logical_mb": logical / 1e6, "unique_mb": unique / 1e6}
+            "logical_mb": logical / 1e6, "unique_mb": unique / 1e6,
+            "shared_prefix_call": {"us_per_layer": us_shared,
+                                   "logical_gb_per_s": logical / (us_shared * 1e-6) / 1e9,
+                                   "unique_gb_per_s": unique / (us_shared * 1e-6) / 1e9}}
 
 
 def large_serving_measurement(reps: int = 12):

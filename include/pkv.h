@@ -219,6 +219,46 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
                                int32_t out_dtype, void* workspace, size_t workspace_bytes,
                                pkv_stream_t stream);
 
+/* Shared-prefix decode attention: the same result as pkv_paged_decode_attn
+ * for requests forked from common prompts, reading each shared block once
+ * per group instead of once per request.  Forked requests share the full
+ * blocks of their prompt by reference ([P2] section "只读时共用，要写入时再分开");
+ * attention still covers each request's whole history ([P2] section
+ * "分页以后，attention 仍然按完整历史归一化"), split into the shared part and
+ * the request's own part, whose online-softmax states merge exactly ([P2]
+ * exercise "逻辑顺序没错，为什么 attention 输出还是错？").
+ *   group_start   DEVICE int32 [num_groups + 1]: group g is the requests
+ *                 group_start[g] .. group_start[g+1]-1 (consecutive rows);
+ *                 group_start[0] = 0, group_start[num_groups] = num_seqs;
+ *                 every request is in exactly one group (a group of one with
+ *                 no shared blocks is plain decode)
+ *   prefix_blocks DEVICE int32 [num_groups]: the first prefix_blocks[g]
+ *                 entries of every member's table row are the same full
+ *                 blocks; every member's length is at least
+ *                 prefix_blocks[g] * block_size
+ *   max_group     largest group size, 1..16, with G * max_group <= 16
+ *                 (G = num_q_heads / num_kv_heads)
+ *   workspace     at least pkv_shared_prefix_workspace_bytes(...) bytes,
+ *                 256-byte aligned; pkv_decode_status(workspace) reports
+ *                 device-detected faults, including members whose table rows
+ *                 differ inside the shared part or groups that break the
+ *                 rules above (PKV_ERR_BAD_TABLE: the output is then not
+ *                 meaningful)
+ * Other arguments as pkv_paged_decode_attn.  Six launches: a gather, two
+ * plans, the shared-part pass (the members' queries are the columns of one
+ * launch), the own-part pass, and the combine. */
+size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t max_blocks_per_seq);
+int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t num_seqs, const int32_t* group_start,
+                                        const int32_t* prefix_blocks, int32_t num_groups, int32_t max_group,
+                                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t block_size, int32_t num_blocks, float scale, int32_t kv_dtype,
+                                        void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                        pkv_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace status word, clears it and
  * returns PKV_OK, PKV_ERR_BAD_TABLE, PKV_ERR_DEVICE_TIMEOUT or
  * PKV_ERR_PLAN_MISMATCH (the first recorded), or PKV_ERR_CUDA. */

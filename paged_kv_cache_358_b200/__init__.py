@@ -19,7 +19,7 @@ __all__ = [
     "BF16", "F32",
     "decode_workspace_bytes", "paged_decode_attn", "decode_plan", "paged_decode_attn_run",
     "decode_status", "set_decode_kernel", "set_launch_overlap", "paged_decode_attn_append_run",
-    "paged_attn_multi_query",
+    "paged_attn_multi_query", "paged_decode_attn_shared_prefix", "shared_prefix_workspace",
     "kv_append", "block_copy", "slot_mapping", "swap_blocks",
     "BlockAllocator",
 ]
@@ -83,6 +83,10 @@ _SIGS = {
     "pkv_multi_query_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "pkv_paged_attn_multi_query": (ctypes.c_int, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                   _i32, _i32, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
+    "pkv_shared_prefix_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "pkv_paged_decode_attn_shared_prefix": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
+                                                           _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp,
+                                                           _i32, _vp, _sz, _vp]),
     "pkv_set_decode_kernel": (ctypes.c_int, [_i32]),
     "pkv_set_launch_overlap": (ctypes.c_int, [_i32]),
     "pkv_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_ulonglong, _vp, _sz, _vp]),
@@ -231,6 +235,42 @@ def paged_attn_multi_query(q, k_pool, v_pool, block_tables, seq_lens, scale: flo
         _dtype_code(k_pool), _dev(out, "out"), _dtype_code(out), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "paged_attn_multi_query")
+    return out
+
+
+def shared_prefix_workspace(num_seqs: int, num_groups: int, max_group: int, num_q_heads: int,
+                            num_kv_heads: int, head_dim: int, max_blocks: int, device=None):
+    torch = _torch()
+    n = lib().pkv_shared_prefix_workspace_bytes(num_seqs, num_groups, max_group, num_q_heads, num_kv_heads,
+                                                head_dim, max_blocks)
+    if n == 0:
+        raise PkvError(Status.INVALID, "shared_prefix_workspace_bytes")
+    return torch.zeros(int(n), dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_decode_attn_shared_prefix(q, k_pool, v_pool, block_tables, seq_lens, group_start, prefix_blocks,
+                                    max_group: int, scale: float, out=None, out_dtype=None, workspace=None,
+                                    stream=None):
+    """Decode attention for groups of consecutive requests that share the first
+    prefix_blocks[g] blocks of their tables; equal to paged_decode_attn."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    S, Hq, Hkv, D, B, N = _attn_args(q, k_pool, v_pool, block_tables, seq_lens, out)
+    if group_start.dtype != torch.int32 or prefix_blocks.dtype != torch.int32:
+        raise TypeError("group_start and prefix_blocks must be int32")
+    NG = prefix_blocks.shape[0]
+    if group_start.shape[0] != NG + 1:
+        raise ValueError("group_start must have num_groups + 1 entries")
+    if workspace is None:
+        workspace = shared_prefix_workspace(S, NG, max_group, Hq, Hkv, D, block_tables.shape[1], q.device)
+    rc = lib().pkv_paged_decode_attn_shared_prefix(
+        _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens"), S, _dev(group_start, "group_start"),
+        _dev(prefix_blocks, "prefix_blocks"), NG, int(max_group), Hq, Hkv, D, B, N, float(scale),
+        _dtype_code(k_pool), _dev(out, "out"), _dtype_code(out), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "paged_decode_attn_shared_prefix")
     return out
 
 

@@ -297,7 +297,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
-             int32_t num_q_tokens = 1, bool overlap = false) {
+             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -336,6 +336,8 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.out_dtype = out_dtype;
   args.num_workers = geo.NW;
   args.num_q_tokens = num_q_tokens;
+  args.causal = causal;
+  args.lse = lse;
   geo.overlap = overlap;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
@@ -430,6 +432,227 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
   return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                   num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
                   workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, num_q_tokens);
+}
+
+}  // extern "C"
+
+// ===========================================================================
+// Shared-prefix decode attention
+// ===========================================================================
+// Requests forked from one prompt share its full blocks (the same physical
+// ids lead their block tables).  Decode attention over the whole history is
+// split at the end of the shared part into two disjoint token ranges whose
+// results combine exactly (the merge of online-softmax states):
+//   prefix pass: per group, the members' queries are the columns of one
+//     multi-token launch (no causal mask) over the shared blocks, so each
+//     shared K/V tile is read once for the whole group; it writes o_p and
+//     the log-sum-exp lse_p of every (member, head);
+//   suffix pass: per request, plain decode over its own blocks after the
+//     prefix (o_s, lse_s);
+//   combine: out = (2^(lse_p - M) o_p + 2^(lse_s - M) o_s) / (2^(lse_p - M) +
+//     2^(lse_s - M)), M = max(lse_p, lse_s); both empty gives 0.
+// A gather kernel builds the grouped queries, the group and suffix tables and
+// lengths in the workspace, and checks that members agree on the shared ids.
+namespace {
+
+struct CascadeLayout {
+  size_t suf_ws = 0, pre_ws = 0, q_grp = 0, grp_table = 0, grp_len = 0, suf_table = 0, suf_len = 0;
+  size_t o_p = 0, lse_p = 0, o_s = 0, lse_s = 0, total = 0;
+  Geometry gs, gp;
+  bool ok = false;
+};
+
+CascadeLayout cascade_layout(int32_t S, int32_t NG, int32_t T, int32_t Hq, int32_t Hkv, int32_t D, int32_t dtype,
+                             int32_t max_blocks) {
+  CascadeLayout c;
+  const int32_t hq_eff = multi_query_heads(T, Hq, Hkv);
+  if (S < 0 || NG < 0 || max_blocks < 0 || hq_eff <= 0) return c;
+  if (!geometry(S, Hq, Hkv, D, dtype, &c.gs) || !geometry(NG, hq_eff, Hkv, D, dtype, &c.gp)) return c;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t es = dtype == PKV_BF16 ? 2 : 4;
+  size_t o = 0;
+  c.suf_ws = o;  o += up(c.gs.lay.total);        // first: its status word is the call's
+  c.pre_ws = o;  o += up(c.gp.lay.total);
+  c.q_grp = o;  o += up(es * size_t(NG) * T * Hq * D);
+  c.grp_table = o;  o += up(4 * size_t(NG) * max_blocks);
+  c.grp_len = o;  o += up(4 * size_t(NG));
+  c.suf_table = o;  o += up(4 * size_t(S) * max_blocks);
+  c.suf_len = o;  o += up(4 * size_t(S));
+  c.o_p = o;  o += up(4 * size_t(NG) * T * Hq * D);
+  c.lse_p = o;  o += up(4 * size_t(NG) * T * Hq);
+  c.o_s = o;  o += up(4 * size_t(S) * Hq * D);
+  c.lse_s = o;  o += up(4 * size_t(S) * Hq);
+  c.total = o;
+  c.ok = true;
+  return c;
+}
+
+}  // namespace
+
+namespace pkv {
+
+// One block per request s: its group g and member index i, its row of the
+// grouped queries, its suffix table and length; the group's first member also
+// writes the group table and length and zeroes the unused member rows.
+__global__ void cascade_gather_kernel(const char* __restrict__ q, const int32_t* __restrict__ tables,
+                                      int32_t max_blocks, const int32_t* __restrict__ seq_lens, int32_t S,
+                                      const int32_t* __restrict__ group_start,
+                                      const int32_t* __restrict__ prefix_blocks, int32_t NG, int32_t T,
+                                      int32_t row_bytes, int32_t B, char* __restrict__ q_grp,
+                                      int32_t* __restrict__ grp_table, int32_t* __restrict__ grp_len,
+                                      int32_t* __restrict__ suf_table, int32_t* __restrict__ suf_len,
+                                      uint32_t* __restrict__ status) {
+  const int s = blockIdx.x;
+  // group of s: the last g with group_start[g] <= s
+  int lo = 0, hi = NG - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (group_start[mid] <= s) lo = mid; else hi = mid - 1;
+  }
+  const int g = lo;
+  const int first = group_start[g], size = group_start[g + 1] - first;
+  const int i = s - first;
+  const int pb = prefix_blocks[g];
+  const bool bad = i < 0 || i >= size || size > T || pb < 0 || pb > max_blocks ||
+                   seq_lens[s] < pb * B;
+  if (bad) {
+    if (threadIdx.x == 0) record_status(status, kStatusBadTable);
+  }
+  const int pbs = bad ? 0 : pb;
+  const int mi = (i >= 0 && i < T) ? i : 0;
+  // query row: q[s] -> q_grp[g][mi]
+  const uint4* src = reinterpret_cast<const uint4*>(q + size_t(s) * row_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(q_grp + (size_t(g) * T + mi) * row_bytes);
+  for (int u = threadIdx.x; u < row_bytes / 16; u += blockDim.x) dst[u] = src[u];
+  const int32_t* row = tables + size_t(s) * max_blocks;
+  const int32_t* lead = tables + size_t(first) * max_blocks;
+  for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) {
+    suf_table[size_t(s) * max_blocks + j] = j + pbs < max_blocks ? row[j + pbs] : -1;
+    if (j < pbs && row[j] != lead[j]) record_status(status, kStatusBadTable);  // not shared after all
+  }
+  if (threadIdx.x == 0) suf_len[s] = seq_lens[s] - pbs * B;
+  if (i == 0) {
+    for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) grp_table[size_t(g) * max_blocks + j] = row[j];
+    if (threadIdx.x == 0) grp_len[g] = pbs * B;
+    for (int m = size; m < T; ++m) {
+      uint4* z = reinterpret_cast<uint4*>(q_grp + (size_t(g) * T + m) * row_bytes);
+      for (int u = threadIdx.x; u < row_bytes / 16; u += blockDim.x) z[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// One warp per (request, query head): combine the two partial results.
+__global__ void cascade_combine_kernel(const float* __restrict__ o_p, const float* __restrict__ lse_p,
+                                       const float* __restrict__ o_s, const float* __restrict__ lse_s,
+                                       const int32_t* __restrict__ group_start, int32_t NG, int32_t T,
+                                       int32_t S, int32_t Hq, int32_t D, void* out, int32_t out_dtype,
+                                       uint32_t* __restrict__ status, const uint32_t* __restrict__ pre_status) {
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid == 0 && lane == 0 && *pre_status) record_status(status, *pre_status);
+  if (wid >= static_cast<long long>(S) * Hq) return;
+  const int s = static_cast<int>(wid / Hq), h = static_cast<int>(wid % Hq);
+  int lo = 0, hi = NG - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (group_start[mid] <= s) lo = mid; else hi = mid - 1;
+  }
+  int i = s - group_start[lo];
+  i = i < 0 ? 0 : (i >= T ? T - 1 : i);
+  const size_t pr = (static_cast<size_t>(lo) * T + i) * Hq + h;  // prefix row
+  const size_t sr = static_cast<size_t>(s) * Hq + h;              // suffix row
+  const float lp = lse_p[pr], ls = lse_s[sr];
+  const float M = fmaxf(lp, ls);
+  float wp = 0.f, wsf = 0.f;
+  if (M != -INFINITY) {
+    wp = exp2f(lp - M);
+    wsf = exp2f(ls - M);
+  }
+  const float den = wp + wsf;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  for (int d = lane; d < D; d += 32) {
+    const float v = (wp * o_p[pr * D + d] + wsf * o_s[sr * D + d]) * inv;
+    store1(out, out_dtype, sr * D + d, v);
+  }
+}
+
+}  // namespace pkv
+
+extern "C" {
+
+size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t max_blocks_per_seq) {
+  size_t best = 0;
+  for (int dt : {PKV_BF16, PKV_F32}) {
+    const CascadeLayout c = cascade_layout(num_seqs, num_groups, max_group, num_q_heads, num_kv_heads, head_dim,
+                                           dt, max_blocks_per_seq);
+    if (c.ok && c.total > best) best = c.total;
+  }
+  return best;
+}
+
+int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t num_seqs, const int32_t* group_start,
+                                        const int32_t* prefix_blocks, int32_t num_groups, int32_t max_group,
+                                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t block_size, int32_t num_blocks, float scale, int32_t kv_dtype,
+                                        void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                        pkv_stream_t stream) {
+  if (num_seqs < 0 || num_groups < 0 || (num_seqs > 0 && num_groups < 1) || num_groups > num_seqs ||
+      max_group < 1 || max_group > 16)
+    return PKV_ERR_INVALID;
+  const CascadeLayout c = cascade_layout(num_seqs, num_groups, max_group, num_q_heads, num_kv_heads, head_dim,
+                                         kv_dtype, max_blocks_per_seq);
+  if (!c.ok) return PKV_ERR_INVALID;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < c.total) return PKV_ERR_INVALID;
+  int rc = check_common(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, block_size,
+                        num_blocks, out, out_dtype, workspace, c.gs.lay.total, c.gs);
+  if (rc != PKV_OK) return rc;
+  if (!std::isfinite(scale)) return PKV_ERR_INVALID;
+  if (num_seqs == 0) return PKV_OK;
+  if (!group_start || !prefix_blocks) return PKV_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  const int32_t row_bytes = num_q_heads * head_dim * (kv_dtype == PKV_BF16 ? 2 : 4);
+  // The suffix workspace leads: clear its status word, the call's own.
+  cudaError_t e = cudaMemsetAsync(w + c.suf_ws, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return host::cuda_fail(e);
+  cascade_gather_kernel<<<num_seqs, 128, 0, st>>>(
+      static_cast<const char*>(q), block_tables, max_blocks_per_seq, seq_lens, num_seqs, group_start,
+      prefix_blocks, num_groups, max_group, row_bytes, block_size, w + c.q_grp,
+      reinterpret_cast<int32_t*>(w + c.grp_table), reinterpret_cast<int32_t*>(w + c.grp_len),
+      reinterpret_cast<int32_t*>(w + c.suf_table), reinterpret_cast<int32_t*>(w + c.suf_len),
+      reinterpret_cast<uint32_t*>(w + c.suf_ws));
+  rc = host::check_launch();
+  if (rc != PKV_OK) return rc;
+  // prefix pass: groups x members, every member sees the whole shared part
+  rc = do_plan(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws, st);
+  if (rc != PKV_OK) return rc;
+  rc = run_impl(w + c.q_grp, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.grp_table),
+                max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
+                num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
+                w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, false, 0,
+                reinterpret_cast<float*>(w + c.lse_p));
+  if (rc != PKV_OK) return rc;
+  // suffix pass: each request over its own blocks
+  rc = do_plan(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws, st);
+  if (rc != PKV_OK) return rc;
+  rc = run_impl(q, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.suf_table), max_blocks_per_seq,
+                reinterpret_cast<const int32_t*>(w + c.suf_len), num_seqs, num_q_heads, num_kv_heads, head_dim,
+                block_size, num_blocks, scale, kv_dtype, w + c.o_s, PKV_F32, w + c.suf_ws, c.gs.lay.total,
+                stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
+  if (rc != PKV_OK) return rc;
+  const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
+  const int threads = 256;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  cascade_combine_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+      reinterpret_cast<const float*>(w + c.o_p), reinterpret_cast<const float*>(w + c.lse_p),
+      reinterpret_cast<const float*>(w + c.o_s), reinterpret_cast<const float*>(w + c.lse_s), group_start,
+      num_groups, max_group, num_seqs, num_q_heads, head_dim, out, out_dtype,
+      reinterpret_cast<uint32_t*>(w + c.suf_ws), reinterpret_cast<const uint32_t*>(w + c.pre_ws));
+  return host::check_launch();
 }
 
 int pkv_decode_status(void* workspace, pkv_stream_t stream) {

@@ -86,7 +86,12 @@ struct DecodeArgs {
   int32_t out_dtype;
   int32_t num_workers;
   int32_t num_q_tokens;  // T query tokens per request (1 for plain decode)
+  int32_t causal;        // T > 1: 1 = token i sees positions < len - (T-1-i); 0 = all see all
   float scale_log2;     // scale * log2(e)
+  // Optional log-sum-exp output (null: none): lse[s][i][h] = log2 of the
+  // softmax denominator in the log2 domain of the scores (-inf when nothing
+  // was attended), for combining this result with another over other tokens.
+  float* lse;
   // Folded append (all null when the new tokens were appended separately):
   // row s of k_new / v_new is request s's new token, the last of its history,
   // written to pool slot new_slots[s] (< 0: no new token for s).
@@ -127,10 +132,12 @@ struct TileLim {
   int rem;     // length - first position of the tile (may exceed 16)
   int T;       // query tokens per request
   int Gq;      // grouped query heads per KV head
+  int causal_on;  // 0: the T tokens all see the whole history (columns differ only in q)
   PKV_DEVINL int lim(int c) const {
     if constexpr (!kCausal) {
       return nvalid;
     } else {
+      if (!causal_on) return nvalid;
       const int causal_lim = rem - (T - 1 - c / Gq);
       return causal_lim < nvalid ? causal_lim : nvalid;
     }
@@ -150,6 +157,11 @@ struct OutMap {
   PKV_DEVINL size_t row(int c) const {
     if (ncols == Gq) return row0 + static_cast<size_t>(c) * D;  // one token: rows are adjacent
     return row0 + static_cast<size_t>(c / Gq) * tok_stride + static_cast<size_t>(c % Gq) * D;
+  }
+  // Optional log-sum-exp output (lse null: none), one value per output row:
+  // log2 of the softmax denominator of column c from its running max m and sum l.
+  PKV_DEVINL void put_lse(float* lse, int c, float m, float l) const {
+    if (lse != nullptr && c < ncols) lse[row(c) / static_cast<size_t>(D)] = l > 0.f ? m + __log2f(l) : -INFINITY;
   }
 };
 

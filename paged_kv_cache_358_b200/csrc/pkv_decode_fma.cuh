@@ -226,7 +226,7 @@ struct FmaCore {
   // Reduce the warp's state and write either the final output (complete
   // pair) or a partial state (o[G][D], m[G], l[G]) for the merge kernel.
   static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype,
-                                const OutMap& om, float* part, int lane) {
+                                const OutMap& om, float* part, int lane, float* lse = nullptr) {
     const int u = lane & (U - 1);
     const int tg = lane >> LOGU;
 #pragma unroll
@@ -245,6 +245,13 @@ struct FmaCore {
       mk[k] = __shfl_sync(0xffffffffu, st.m, k * LPH);
     }
     if (complete) {
+      if (lane < G) {
+        float ml = mk[0], ll = lk[0];
+#pragma unroll
+        for (int k = 1; k < G; ++k)
+          if (lane == k) ml = mk[k], ll = lk[k];
+        om.put_lse(lse, lane, ml, ll);
+      }
       if (tg == 0) {
 #pragma unroll
         for (int k = 0; k < G; ++k) {

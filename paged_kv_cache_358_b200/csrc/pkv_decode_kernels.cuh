@@ -22,6 +22,11 @@ namespace pkv {
 // Lanes read the (CTA, head) states of a pass together, so the merge costs a
 // couple of memory round trips, not one per CTA.
 // ---------------------------------------------------------------------------
+// The log-sum-exp output of a general (MULTI) launch, for the merge: passing
+// it as one more argument would change the register allocation of the
+// streaming loop around the call.
+__shared__ float* s_lse_out;
+
 // Kept out of line: its load batches need many registers for a moment, and
 // inlined they would raise the register count of the whole streaming loop.
 template <int D, int G, int HG, bool MULTI>
@@ -100,6 +105,9 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
       }
     }
   }
+  if constexpr (MULTI) {  // lane k holds column k's running max and sum
+    if (lane < G) om.put_lse(s_lse_out, lane, run_m, run_l);
+  }
 #pragma unroll
   for (int k = 0; k < G; ++k) {
     const float lk = __shfl_sync(0xffffffffu, run_l, k);
@@ -153,9 +161,9 @@ struct TmaMaps {
   CUtensorMap v;
 };
 
-// MULTI: several query tokens per request (causal) or idle padding columns;
-// without it the columns are exactly the G grouped heads of one token and the
-// kernel has no per-column work.
+// MULTI: several query tokens per request, idle padding columns, or a
+// log-sum-exp output; without it the columns are exactly the G grouped heads
+// of one token and the kernel has no per-column work.
 template <class Core, int G, int W, int CPS, int DEPTH, bool MULTI>
 __global__ void __launch_bounds__(W * 32, CPS)
     partition_kernel(const __grid_constant__ TmaMaps maps, const DecodeArgs a, int check_S,
@@ -216,6 +224,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
       for (int i = ncols * Core::ROWB / 16 + lane; i < Core::QB / 16; i += 32)
         reinterpret_cast<uint4*>(stages + st * Core::kStageBytes + Core::kQOff)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
+  }
+  if constexpr (MULTI) {
+    if (threadIdx.x == 0) s_lse_out = a.lse;
   }
   if (ntiles > 0 && lane == 0) {
     for (int i = 0; i < DEPTH; ++i) mbar_init(smem_u32(&bars[i]), 1);
@@ -416,6 +427,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const OutMap om{(static_cast<size_t>(s) * T * Hq + static_cast<size_t>(hg * W + warp) * Gq) * D,
                     static_cast<size_t>(Hq) * D, Gq, D, ncols};
     for (int i = lane; i < ncols * D; i += 32) store1(a.out, a.out_dtype, om.row(i / D) + i % D, 0.f);
+    if constexpr (MULTI) {
+      if (lane < ncols) om.put_lse(a.lse, lane, -INFINITY, 0.f);
+    }
   }
   if (ntiles <= 0) return;
 
@@ -429,8 +443,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const int head = phg * W + warp;
     const OutMap om{(static_cast<size_t>(ps) * T * Hq + static_cast<size_t>(head) * Gq) * D,
                     static_cast<size_t>(Hq) * D, Gq, D, ncols};
+    float* const lse = MULTI ? a.lse : nullptr;
     if (jfirst == 0 && last_is_end) {  // the whole pair is in this CTA's range
-      Core::finish(state, true, a.out, a.out_dtype, om, nullptr, lane);
+      Core::finish(state, true, a.out, a.out_dtype, om, nullptr, lane, lse);
       return;
     }
     const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
@@ -495,7 +510,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       }
       __syncwarp();
     }
-    const TileLim<MULTI> lim{nvalid, MULTI ? m.len - m.j * kTile : nvalid, T, Gq};
+    const TileLim<MULTI> lim{nvalid, MULTI ? m.len - m.j * kTile : nvalid, T, Gq, a.causal};
     if constexpr (Core::kSwizzle) {
       Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, lim, a.scale_log2, lane);
     } else {
@@ -571,7 +586,7 @@ int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, cons
                 cudaStream_t stream) {
   constexpr int WPS = (Core::ROWB >= 512) ? 4 : 8;
   if (geo.HG != 1) return PKV_ERR_INVALID;
-  if (args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads)
+  if (args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads || args.lse != nullptr)
     return launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream);
   return launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
 }

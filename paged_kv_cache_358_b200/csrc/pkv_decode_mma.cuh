@@ -231,7 +231,7 @@ struct MmaCore {
   }
 
   static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, const OutMap& om,
-                                float* part, int lane) {
+                                float* part, int lane, float* lse = nullptr) {
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
@@ -244,6 +244,10 @@ struct MmaCore {
       const int h0 = 8 * nb + 2 * tig, h1 = h0 + 1;
       if (complete) {
         const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;  // 0: nothing attended
+        if (gid == 0) {
+          om.put_lse(lse, h0, st.m[nb][0], l0);
+          om.put_lse(lse, h1, st.m[nb][1], l1);
+        }
         const size_t r0 = om.row(h0), r1 = om.row(h1);
 #pragma unroll
         for (int mt = 0; mt < KSTEPS; ++mt) {
