@@ -136,3 +136,20 @@ def test_shared_prefix_flags_a_false_claim():
                                         torch.from_numpy(lens).cuda(), torch.from_numpy(gs).cuda(),
                                         torch.from_numpy(pb).cuda(), 2, 1.0 / np.sqrt(D), workspace=ws)
     assert pkv.decode_status(ws) == pkv.Status.BAD_TABLE
+
+
+def test_shared_prefix_rejects_unsupported_groups():
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    L = pkv.lib()
+    assert L.pkv_shared_prefix_workspace_bytes(8, 2, 4, 16, 4, 128, 10) > 0
+    assert L.pkv_shared_prefix_workspace_bytes(8, 2, 5, 16, 4, 128, 10) == 0     # 5 x 4 columns > 16
+    assert L.pkv_shared_prefix_workspace_bytes(8, 2, 17, 8, 8, 128, 10) == 0     # more than 16 members
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = L.pkv_paged_decode_attn_shared_prefix(z.data_ptr(), z.data_ptr(), z.data_ptr(), z.data_ptr(), 1,
+                                               z.data_ptr(), 4, z.data_ptr(), z.data_ptr(), 5, 2, 16, 4, 128,
+                                               16, 1, 0.1, pkv.BF16, z.data_ptr(), pkv.BF16, z.data_ptr(), 1 << 20,
+                                               None)
+    assert rc == pkv.Status.INVALID                                              # more groups than requests
