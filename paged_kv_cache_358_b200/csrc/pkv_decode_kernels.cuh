@@ -597,11 +597,15 @@ int run_decode(const Geometry& geo, const DecodeArgs& args, const void* k, const
                cudaStream_t stream) {
   auto per_g = [&](auto gc) -> int {
     constexpr int G = decltype(gc)::value;
-    // tensor-core tiles for bf16: up to 16 columns at head_dim <= 128 (two
-    // 8-column blocks), up to 8 at head_dim 256 (their registers run out)
-    if constexpr (sizeof(T) == 2 && (G <= 8 || D <= 128)) {
+    // tensor-core tiles for bf16: up to 8 columns with the tokens in the MMA's
+    // M dimension; 16 columns (head_dim <= 128) with the columns in M
+    if constexpr (sizeof(T) == 2 && G <= 8) {
       if (args.block_size >= 8 && g_kernel_choice != 1)
         return launch_core<MmaCore<D, G>, G>(geo, args, k, v, stream);
+    }
+    if constexpr (sizeof(T) == 2 && G == 16 && D <= 128) {
+      if (args.block_size >= 8 && g_kernel_choice != 1)
+        return launch_core<MmaCoreM16<D>, G>(geo, args, k, v, stream);
     }
     return launch_core<FmaCore<T, D, G>, G>(geo, args, k, v, stream);
   };

@@ -296,4 +296,205 @@ struct MmaCore {
   }
 };
 
+// Tensor-core core for 16 grouped columns (G = 16, or T query tokens x Gq
+// heads = 16), with the columns in the MMA's M dimension:
+//   scores  S[16 cols x 16 tok] = Q[16 x D] * K^T[D x 16]   (2 * D/16 MMAs)
+//   values  O[16 cols x D]     += P[16 x 16 tok] * V[16 tok x D] (D/8 MMAs)
+// The score accumulators of the two 8-token halves are, packed to bf16,
+// exactly the A operand of the value product (no transpose), and a column's
+// 16 scores sit in the 4 lanes of one quad (2 shuffle levels for its max and
+// sum).  K is read with ldmatrix as the B operand, V with ldmatrix.trans.
+// Same shared-memory stage layout as MmaCore (TMA 128-byte swizzle).
+template <int D>
+struct MmaCoreM16 {
+  using Base = MmaCore<D, 16>;
+  static constexpr int G = 16;
+  static constexpr int ESZ = Base::ESZ;
+  static constexpr int ROWB = Base::ROWB;
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int NT = D / 8;  // 8-wide output column tiles
+  static constexpr int QB = Base::QB;
+  static constexpr int kAlign = Base::kAlign;
+  static constexpr int kKOff = Base::kKOff;
+  static constexpr int kVOff = Base::kVOff;
+  static constexpr int kQOff = Base::kQOff;
+  static constexpr int kStageBytes = Base::kStageBytes;
+  static constexpr int kChunks = Base::kChunks;
+  static constexpr int kBoxInner = Base::kBoxInner;
+  static constexpr int kChunkRowBytes = Base::kChunkRowBytes;
+  static constexpr int kChunkBytes = Base::kChunkBytes;
+  static constexpr bool kSwizzle = true;
+  static constexpr int kScratchBytes = 0;
+  static_assert(D <= 128, "the 16-row accumulator of head_dim 256 does not fit the registers");
+
+  struct State {
+    uint32_t qa[KSTEPS][4];  // Q A-fragments: rows gid / gid+8, k = 2tig(+1) / 2tig+8(+9)
+    float o[NT][4];          // O rows gid / gid+8, cols 8*nt + 2tig (+1)
+    float m[2];              // running max of rows gid, gid+8 (log2 domain; equal over a quad)
+    float l[2];              // this lane's share of the running sums
+  };
+
+  static PKV_DEVINL uint32_t swz(int t, int unit) { return Base::swz(t, unit); }
+  static PKV_DEVINL uint32_t row_unit(int t, int unit) { return Base::swz(t, unit); }
+
+  static PKV_DEVINL void begin_pair(State& st, const char* qsm, float /*scale_log2*/, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const char* r0 = qsm + gid * ROWB + (16 * kk + 2 * tig) * 2;
+      const char* r1 = r0 + 8 * ROWB;
+      st.qa[kk][0] = *reinterpret_cast<const uint32_t*>(r0);
+      st.qa[kk][1] = *reinterpret_cast<const uint32_t*>(r1);
+      st.qa[kk][2] = *reinterpret_cast<const uint32_t*>(r0 + 16);
+      st.qa[kk][3] = *reinterpret_cast<const uint32_t*>(r1 + 16);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) st.o[nt][0] = st.o[nt][1] = st.o[nt][2] = st.o[nt][3] = 0.f;
+    st.m[0] = st.m[1] = -INFINITY;
+    st.l[0] = st.l[1] = 0.f;
+  }
+
+  template <class Lim>
+  static PKV_DEVINL void tile(State& st, const char* ksm, const char* vsm, const Lim& L, float scale_log2,
+                              int lane) {
+    const int nvalid = L.nvalid;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
+
+    // scores: s0 for tokens 0..7, s1 for tokens 8..15 (C rows = columns)
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      // matrices: (tok 0-7, unit 2kk), (tok 0-7, 2kk+1), (tok 8-15, 2kk), (tok 8-15, 2kk+1)
+      const int t = (lane & 7) + ((lane >> 4) << 3);
+      const int hu = (lane >> 3) & 1;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + swz(t, 2 * kk + hu), b0, b1, b2, b3);
+        mma_bf16_16816(s0, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b0, b1);
+        mma_bf16_16816(s1, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b2, b3);
+      }
+    }
+    // row gid: s0[0], s0[1], s1[0], s1[1] (tokens 2tig, 2tig+1, 8+2tig, 9+2tig); row gid+8: [2], [3]
+    const int lim0 = L.lim(gid), lim1 = L.lim(gid + 8);
+    const int t0 = 2 * tig;
+    float x[8];
+    x[0] = t0 < lim0 ? s0[0] * scale_log2 : -INFINITY;
+    x[1] = t0 + 1 < lim0 ? s0[1] * scale_log2 : -INFINITY;
+    x[2] = t0 + 8 < lim0 ? s1[0] * scale_log2 : -INFINITY;
+    x[3] = t0 + 9 < lim0 ? s1[1] * scale_log2 : -INFINITY;
+    x[4] = t0 < lim1 ? s0[2] * scale_log2 : -INFINITY;
+    x[5] = t0 + 1 < lim1 ? s0[3] * scale_log2 : -INFINITY;
+    x[6] = t0 + 8 < lim1 ? s1[2] * scale_log2 : -INFINITY;
+    x[7] = t0 + 9 < lim1 ? s1[3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    float mx1 = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
+#pragma unroll
+    for (int msk = 1; msk < 4; msk <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+    }
+    const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+    float r0 = mn0, r1 = mn1;
+    if constexpr (Lim::causal) {  // a column with no valid score yet: subtract 0, not -inf
+      r0 = mn0 == -INFINITY ? 0.f : mn0;
+      r1 = mn1 == -INFINITY ? 0.f : mn1;
+    }
+    const float al0 = exp2f(st.m[0] - r0), al1 = exp2f(st.m[1] - r1);
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      p[i] = exp2f(x[i] - r0);
+      p[4 + i] = exp2f(x[4 + i] - r1);
+    }
+    st.l[0] = st.l[0] * al0 + ((p[0] + p[1]) + (p[2] + p[3]));
+    st.l[1] = st.l[1] * al1 + ((p[4] + p[5]) + (p[6] + p[7]));
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        st.o[nt][0] *= al0;
+        st.o[nt][1] *= al0;
+        st.o[nt][2] *= al1;
+        st.o[nt][3] *= al1;
+      }
+    }
+    // P as the A operand: rows gid / gid+8, tokens 2tig(+1) and 8+2tig(+1)
+    const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
+    const uint32_t pa1 = pack_bf16x2(p[4], p[5]);
+    const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
+    const uint32_t pa3 = pack_bf16x2(p[6], p[7]);
+
+    // values: V as the B operand via ldmatrix.trans; matrices (tok 0-7, unit
+    // 2mt), (tok 8-15, 2mt), (tok 0-7, 2mt+1), (tok 8-15, 2mt+1)
+    const int vt = (lane & 7) + (((lane >> 3) & 1) << 3);
+    const int vu = lane >> 4;
+    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+    const bool tail = nvalid < kTile;
+    if (tail) {  // V rows at or past the length never reach the accumulator (0 * NaN)
+      mlo = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+      mhi = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(vbase + swz(vt, 2 * mt + vu), b0, b1, b2, b3);
+      if (tail) {
+        b0 &= mlo;
+        b1 &= mhi;
+        b2 &= mlo;
+        b3 &= mhi;
+      }
+      mma_bf16_16816(st.o[2 * mt], pa0, pa1, pa2, pa3, b0, b1);
+      mma_bf16_16816(st.o[2 * mt + 1], pa0, pa1, pa2, pa3, b2, b3);
+    }
+  }
+
+  static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, const OutMap& om,
+                                float* part, int lane, float* lse = nullptr) {
+    const int gid = lane >> 2, tig = lane & 3;
+    float l0 = st.l[0], l1 = st.l[1];
+#pragma unroll
+    for (int msk = 1; msk < 4; msk <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
+    }
+    const int c0 = gid, c1 = gid + 8;
+    if (complete) {
+      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;  // 0: nothing attended
+      if (tig == 0) {
+        om.put_lse(lse, c0, st.m[0], l0);
+        om.put_lse(lse, c1, st.m[1], l1);
+      }
+      const size_t r0 = om.row(c0), r1 = om.row(c1);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int d = 8 * nt + 2 * tig;
+        if (c0 < om.ncols) {
+          Base::put(out, out_dtype, r0 + d, st.o[nt][0] * i0);
+          Base::put(out, out_dtype, r0 + d + 1, st.o[nt][1] * i0);
+        }
+        if (c1 < om.ncols) {
+          Base::put(out, out_dtype, r1 + d, st.o[nt][2] * i1);
+          Base::put(out, out_dtype, r1 + d + 1, st.o[nt][3] * i1);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int d = 8 * nt + 2 * tig;
+        *reinterpret_cast<float2*>(part + c0 * D + d) = make_float2(st.o[nt][0], st.o[nt][1]);
+        *reinterpret_cast<float2*>(part + c1 * D + d) = make_float2(st.o[nt][2], st.o[nt][3]);
+      }
+      if (tig == 0) {
+        part[G * D + c0] = st.m[0];
+        part[G * D + c1] = st.m[1];
+        part[G * D + G + c0] = l0;
+        part[G * D + G + c1] = l1;
+      }
+    }
+  }
+};
+
 }  // namespace pkv
