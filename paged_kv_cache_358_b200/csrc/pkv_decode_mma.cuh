@@ -8,11 +8,10 @@
 // M >= 64 and a TMEM round trip per tile for the softmax; the warp-level
 // m16n8k16 shape fits one 16-token tile and the grouped heads directly.
 //
-// Shapes per 16-token tile (tokens in M, grouped columns in N, in blocks of 8;
-// one block for up to 8 columns, two for up to 16):
-//   scores  S^T[16 tok x 8 cols] = K[16 x D] * Q^T[D x 8]      (D/16 MMAs per block)
-//   values  O^T[D x 8 cols]     += V^T[D x 16 tok] * P^T[16 x 8] (D/16 MMAs per block)
-// The K and V^T fragments of a step are loaded once and used by every block.
+// Shapes per 16-token tile (tokens in M, up to 8 grouped columns in N):
+//   scores  S^T[16 tok x 8 cols] = K[16 x D] * Q^T[D x 8]      (D/16 MMAs)
+//   values  O^T[D x 8 cols]     += V^T[D x 16 tok] * P^T[16 x 8] (D/16 MMAs)
+// (16 columns use MmaCoreM16 below, with the columns in M.)
 // K and V tiles arrive through TMA with the 128-byte swizzle, so ldmatrix
 // (plain for K, .trans for V^T) reads them without bank conflicts.  The
 // score accumulator (token-major) is turned into the P^T operand of the value
@@ -67,7 +66,6 @@ struct MmaCore {
   static constexpr int ROWB = D * ESZ;
   static constexpr int NCH = ROWB / 128;      // 128-byte swizzle atoms per row
   static constexpr int KSTEPS = D / 16;
-  static constexpr int NB = (G + 7) / 8;      // 8-column MMA blocks of grouped columns
   static constexpr int CHUNKB = kTile * 128;  // one swizzled chunk of a tile
   static constexpr int TILEB = NCH * CHUNKB;
   static constexpr int QB = G * ROWB;
@@ -83,14 +81,14 @@ struct MmaCore {
   static constexpr bool kSwizzle = true;
   static constexpr int kScratchBytes = 0;
 
-  static_assert(G >= 1 && G <= 16, "grouped columns must fit two 8-column MMA blocks");
+  static_assert(G >= 1 && G <= 8, "grouped heads must fit the 8 MMA columns");
   static_assert(NCH >= 1 && NCH <= 4, "head_dim 64, 128 or 256");
 
   struct State {
-    uint32_t qb[NB][KSTEPS][2];  // Q^T B-fragments (bf16x2), columns >= G are zero
-    float oc[NB][KSTEPS][4];     // O^T accumulator: rows d = 16*mt + gid (+8), cols 8*nb + 2*tig (+1)
-    float m[NB][2];              // running max of columns 8*nb + 2*tig (+1) (log2 domain)
-    float l[NB][2];              // this lane's share of the running sums
+    uint32_t qb[KSTEPS][2];  // Q^T B-fragments (bf16x2), heads >= G are zero
+    float oc[KSTEPS][4];     // O^T accumulator: rows d = 16*mt + gid (+8), cols heads 2*tig (+1)
+    float m[2];              // running max of heads 2*tig, 2*tig+1 (log2 domain)
+    float l[2];              // this lane's share of the running sums
   };
 
   // Byte offset of (row t, 16-byte unit) inside a swizzled tile.
@@ -104,24 +102,20 @@ struct MmaCore {
   static PKV_DEVINL void begin_pair(State& st, const char* qsm, float /*scale_log2*/, int lane) {
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int col = 8 * nb + gid;
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        if (col < G) {
-          const char* row = qsm + col * ROWB + (16 * kk + 2 * tig) * 2;
-          st.qb[nb][kk][0] = *reinterpret_cast<const uint32_t*>(row);
-          st.qb[nb][kk][1] = *reinterpret_cast<const uint32_t*>(row + 16);
-        } else {
-          st.qb[nb][kk][0] = 0u;
-          st.qb[nb][kk][1] = 0u;
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) st.oc[nb][kk][i] = 0.f;
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      if (gid < G) {
+        const char* row = qsm + gid * ROWB + (16 * kk + 2 * tig) * 2;
+        st.qb[kk][0] = *reinterpret_cast<const uint32_t*>(row);
+        st.qb[kk][1] = *reinterpret_cast<const uint32_t*>(row + 16);
+      } else {
+        st.qb[kk][0] = 0u;
+        st.qb[kk][1] = 0u;
       }
-      st.m[nb][0] = st.m[nb][1] = -INFINITY;
-      st.l[nb][0] = st.l[nb][1] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.oc[kk][i] = 0.f;
     }
+    st.m[0] = st.m[1] = -INFINITY;
+    st.l[0] = st.l[1] = 0.f;
   }
 
   template <class Lim>
@@ -131,10 +125,8 @@ struct MmaCore {
     const int gid = lane >> 2, tig = lane & 3;
     const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
 
-    // scores S^T = K Q^T, one K fragment per k-step shared by the column blocks
-    float c[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0.f;
+    // scores S^T = K Q^T
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
     {
       const int t = lane & 15;
       const int cb = lane >> 4;
@@ -142,71 +134,53 @@ struct MmaCore {
       for (int kk = 0; kk < KSTEPS; ++kk) {
         uint32_t a0, a1, a2, a3;
         ldsm_x4(kbase + swz(t, 2 * kk + cb), a0, a1, a2, a3);
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(c[nb], a0, a1, a2, a3, st.qb[nb][kk][0], st.qb[nb][kk][1]);
+        mma_bf16_16816(c, a0, a1, a2, a3, st.qb[kk][0], st.qb[kk][1]);
       }
     }
-    // c[nb][0]: (tok gid, col 8nb+2tig), [1]: (gid, 8nb+2tig+1), [2]: (gid+8, 8nb+2tig), [3]: (gid+8, 8nb+2tig+1)
-    float p[NB][4];
-    bool rescale = false;
-    float al[NB][2];
+    // c[0]: (tok gid, col 2tig), c[1]: (gid, 2tig+1), c[2]: (gid+8, 2tig), c[3]: (gid+8, 2tig+1)
+    const int lim0 = L.lim(2 * tig), lim1 = L.lim(2 * tig + 1);
+    float s[4];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int lim0 = L.lim(8 * nb + 2 * tig), lim1 = L.lim(8 * nb + 2 * tig + 1);
-      float s[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = gid + ((i & 2) ? 8 : 0);
-        s[i] = t < ((i & 1) ? lim1 : lim0) ? c[nb][i] * scale_log2 : -INFINITY;
-      }
-      float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
-#pragma unroll
-      for (int msk = 4; msk < 32; msk <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
-      }
-      const float mn0 = fmaxf(st.m[nb][0], mx0), mn1 = fmaxf(st.m[nb][1], mx1);
-      // Under the causal mask a column may have seen no valid score yet and
-      // keep m = -inf: subtract 0 instead, so every exponent is exp2(-inf) = 0
-      // and nothing becomes NaN.  Without it every tile has a valid row.
-      float r0 = mn0, r1 = mn1;
-      if constexpr (Lim::causal) {
-        r0 = mn0 == -INFINITY ? 0.f : mn0;
-        r1 = mn1 == -INFINITY ? 0.f : mn1;
-      }
-      al[nb][0] = exp2f(st.m[nb][0] - r0);
-      al[nb][1] = exp2f(st.m[nb][1] - r1);
-      st.m[nb][0] = mn0;
-      st.m[nb][1] = mn1;
-      p[nb][0] = exp2f(s[0] - r0);
-      p[nb][1] = exp2f(s[1] - r1);
-      p[nb][2] = exp2f(s[2] - r0);
-      p[nb][3] = exp2f(s[3] - r1);
-      st.l[nb][0] = st.l[nb][0] * al[nb][0] + (p[nb][0] + p[nb][2]);
-      st.l[nb][1] = st.l[nb][1] * al[nb][1] + (p[nb][1] + p[nb][3]);
-      rescale = rescale || al[nb][0] != 1.f || al[nb][1] != 1.f;
+    for (int i = 0; i < 4; ++i) {
+      const int t = gid + ((i & 2) ? 8 : 0);
+      s[i] = t < ((i & 1) ? lim1 : lim0) ? c[i] * scale_log2 : -INFINITY;
     }
-    if (__any_sync(0xffffffffu, rescale)) {
+    float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          st.oc[nb][mt][0] *= al[nb][0];
-          st.oc[nb][mt][1] *= al[nb][1];
-          st.oc[nb][mt][2] *= al[nb][0];
-          st.oc[nb][mt][3] *= al[nb][1];
-        }
+    for (int msk = 4; msk < 32; msk <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
     }
-
+    const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+    // Under the causal mask a column may have seen no valid score yet and keep
+    // m = -inf: subtract 0 instead, so every exponent is exp2(-inf) = 0 and
+    // nothing becomes NaN.  Without it every tile has a valid row.
+    float r0 = mn0, r1 = mn1;
+    if constexpr (Lim::causal) {
+      r0 = mn0 == -INFINITY ? 0.f : mn0;
+      r1 = mn1 == -INFINITY ? 0.f : mn1;
+    }
+    const float al0 = exp2f(st.m[0] - r0), al1 = exp2f(st.m[1] - r1);
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+    const float p0 = exp2f(s[0] - r0), p1 = exp2f(s[1] - r1);
+    const float p2 = exp2f(s[2] - r0), p3 = exp2f(s[3] - r1);
+    st.l[0] = st.l[0] * al0 + (p0 + p2);
+    st.l[1] = st.l[1] * al1 + (p1 + p3);
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        st.oc[mt][0] *= al0;
+        st.oc[mt][1] *= al1;
+        st.oc[mt][2] *= al0;
+        st.oc[mt][3] *= al1;
+      }
+    }
     // P^T operand: transpose the token-major fragments
-    uint32_t b0[NB], b1[NB];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      b0[nb] = movmatrix_trans(pack_bf16x2(p[nb][0], p[nb][1]));
-      b1[nb] = movmatrix_trans(pack_bf16x2(p[nb][2], p[nb][3]));
-    }
+    const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
 
-    // values O^T += V^T P^T, one V^T fragment per step shared by the column blocks
+    // values O^T += V^T P^T
     const int vt = ((lane >> 4) << 3) + (lane & 7);
     const int vu = (lane >> 3) & 1;
     uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
@@ -225,64 +199,60 @@ struct MmaCore {
         a2 &= mhi;
         a3 &= mhi;
       }
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(st.oc[nb][mt], a0, a1, a2, a3, b0[nb], b1[nb]);
+      mma_bf16_16816(st.oc[mt], a0, a1, a2, a3, b0, b1);
     }
   }
 
   static PKV_DEVINL void finish(State& st, bool complete, void* out, int out_dtype, const OutMap& om,
                                 float* part, int lane, float* lse = nullptr) {
     const int gid = lane >> 2, tig = lane & 3;
+    float l0 = st.l[0], l1 = st.l[1];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      float l0 = st.l[nb][0], l1 = st.l[nb][1];
-#pragma unroll
-      for (int msk = 4; msk < 32; msk <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
+    for (int msk = 4; msk < 32; msk <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
+    }
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+    if (complete) {
+      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;  // 0: nothing attended
+      if (gid == 0) {
+        om.put_lse(lse, h0, st.m[0], l0);
+        om.put_lse(lse, h1, st.m[1], l1);
       }
-      const int h0 = 8 * nb + 2 * tig, h1 = h0 + 1;
-      if (complete) {
-        const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;  // 0: nothing attended
-        if (gid == 0) {
-          om.put_lse(lse, h0, st.m[nb][0], l0);
-          om.put_lse(lse, h1, st.m[nb][1], l1);
-        }
-        const size_t r0 = om.row(h0), r1 = om.row(h1);
+      const size_t r0 = om.row(h0), r1 = om.row(h1);
 #pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          const int d0 = 16 * mt + gid, d1 = d0 + 8;
-          if (h0 < om.ncols) {
-            put(out, out_dtype, r0 + d0, st.oc[nb][mt][0] * i0);
-            put(out, out_dtype, r0 + d1, st.oc[nb][mt][2] * i0);
-          }
-          if (h1 < om.ncols) {
-            put(out, out_dtype, r1 + d0, st.oc[nb][mt][1] * i1);
-            put(out, out_dtype, r1 + d1, st.oc[nb][mt][3] * i1);
-          }
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        if (h0 < om.ncols) {
+          put(out, out_dtype, r0 + d0, st.oc[mt][0] * i0);
+          put(out, out_dtype, r0 + d1, st.oc[mt][2] * i0);
         }
-      } else {
+        if (h1 < om.ncols) {
+          put(out, out_dtype, r1 + d0, st.oc[mt][1] * i1);
+          put(out, out_dtype, r1 + d1, st.oc[mt][3] * i1);
+        }
+      }
+    } else {
 #pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          const int d0 = 16 * mt + gid, d1 = d0 + 8;
-          if (h0 < G) {
-            part[h0 * D + d0] = st.oc[nb][mt][0];
-            part[h0 * D + d1] = st.oc[nb][mt][2];
-          }
-          if (h1 < G) {
-            part[h1 * D + d0] = st.oc[nb][mt][1];
-            part[h1 * D + d1] = st.oc[nb][mt][3];
-          }
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        if (h0 < G) {
+          part[h0 * D + d0] = st.oc[mt][0];
+          part[h0 * D + d1] = st.oc[mt][2];
         }
-        if (gid == 0) {
-          if (h0 < G) {
-            part[G * D + h0] = st.m[nb][0];
-            part[G * D + G + h0] = l0;
-          }
-          if (h1 < G) {
-            part[G * D + h1] = st.m[nb][1];
-            part[G * D + G + h1] = l1;
-          }
+        if (h1 < G) {
+          part[h1 * D + d0] = st.oc[mt][1];
+          part[h1 * D + d1] = st.oc[mt][3];
+        }
+      }
+      if (gid == 0) {
+        if (h0 < G) {
+          part[G * D + h0] = st.m[0];
+          part[G * D + G + h0] = l0;
+        }
+        if (h1 < G) {
+          part[G * D + h1] = st.m[1];
+          part[G * D + G + h1] = l1;
         }
       }
     }
@@ -307,18 +277,18 @@ struct MmaCore {
 // Same shared-memory stage layout as MmaCore (TMA 128-byte swizzle).
 template <int D>
 struct MmaCoreM16 {
-  using Base = MmaCore<D, 16>;
+  using Base = MmaCore<D, 8>;  // tile layout, swizzle and output helpers (independent of G)
   static constexpr int G = 16;
   static constexpr int ESZ = Base::ESZ;
   static constexpr int ROWB = Base::ROWB;
   static constexpr int KSTEPS = D / 16;
   static constexpr int NT = D / 8;  // 8-wide output column tiles
-  static constexpr int QB = Base::QB;
+  static constexpr int QB = G * ROWB;
   static constexpr int kAlign = Base::kAlign;
   static constexpr int kKOff = Base::kKOff;
   static constexpr int kVOff = Base::kVOff;
   static constexpr int kQOff = Base::kQOff;
-  static constexpr int kStageBytes = Base::kStageBytes;
+  static constexpr int kStageBytes = round_up(2 * Base::TILEB + QB, 1024);
   static constexpr int kChunks = Base::kChunks;
   static constexpr int kBoxInner = Base::kBoxInner;
   static constexpr int kChunkRowBytes = Base::kChunkRowBytes;
