@@ -279,6 +279,7 @@ class DecodeStep:
         self.down = torch.cuda.Stream()
         self.e2e_k = 0
         self.in_ready = [None, None]    # per buffer: inputs of its current step on the device
+        self.tables_copied = None       # the last step's table copies are done
         self.step_done = [None, None]   # per buffer: its step's kernels finished
         self.out_back = [None, None]    # per buffer: its step's outputs on the host
 
@@ -323,6 +324,8 @@ class DecodeStep:
         ev = torch.cuda.Event()
         ev.record(self.stream)
         self.h2d_done[b] = ev
+        tables_copied_prev = self.tables_copied
+        self.tables_copied = ev
         if nc:
             pkv.block_copy(self.k_pools, self.v_pools, self.cp_d[:nc])
             self.launches += 1
@@ -333,9 +336,13 @@ class DecodeStep:
         if e2e:
             eb = self.e2e_k % 2
             self.e2e_k += 1
-            # upload this step's inputs once the step that last used the buffer is done
+            # upload this step's inputs once the step that last used the buffer is
+            # done, and after the previous step's small table copies, so those
+            # never queue behind this upload on the copy engine
             if self.step_done[eb] is not None:
                 self.up.wait_event(self.step_done[eb])
+            if tables_copied_prev is not None:
+                self.up.wait_event(tables_copied_prev)
             with torch.cuda.stream(self.up):
                 self.in_d[eb].copy_(self.in_h, non_blocking=True)
             self.in_ready[eb] = torch.cuda.Event()
