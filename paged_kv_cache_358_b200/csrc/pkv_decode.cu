@@ -27,11 +27,16 @@ namespace pkv {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanSmemSeqs = 8192;  // prefix kept in shared memory up to this many requests
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ seq_lens,
-                                                            int S, int Hq, int Hkv, int NHG, int D,
-                                                            int kv_dtype, int NW, char* ws,
-                                                            size_t off_prefix, size_t off_wplan,
-                                                            size_t off_counters) {
+struct PlanArgs {
+  const int32_t* seq_lens;
+  int S, Hq, Hkv, NHG, D, kv_dtype, NW;
+  char* ws;
+  size_t off_prefix, off_wplan, off_counters;
+};
+
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int S, int Hq, int Hkv,
+                                          int NHG, int D, int kv_dtype, int NW, char* ws, size_t off_prefix,
+                                          size_t off_wplan, size_t off_counters) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + off_prefix);
   int4* wplan = reinterpret_cast<int4*>(ws + off_wplan);
@@ -114,6 +119,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     hdr->total_tiles = T;
     hdr->planned = 1;
   }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ seq_lens,
+                                                            int S, int Hq, int Hkv, int NHG, int D,
+                                                            int kv_dtype, int NW, char* ws,
+                                                            size_t off_prefix, size_t off_wplan,
+                                                            size_t off_counters) {
+  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters);
+}
+
+// Two independent plans in one launch, one per CTA.
+__global__ void __launch_bounds__(kPlanThreads) plan2_kernel(const PlanArgs p0, const PlanArgs p1) {
+  const PlanArgs& p = blockIdx.x == 0 ? p0 : p1;
+  plan_body(p.seq_lens, p.S, p.Hq, p.Hkv, p.NHG, p.D, p.kv_dtype, p.NW, p.ws, p.off_prefix, p.off_wplan,
+            p.off_counters);
 }
 
 }  // namespace pkv
@@ -627,22 +647,32 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
       reinterpret_cast<uint32_t*>(w + c.suf_ws));
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
-  // prefix pass: groups x members, every member sees the whole shared part
-  rc = do_plan(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws, st);
+  // both plans in one launch
+  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws) {
+    return PlanArgs{lens, g.S, g.Hq, g.Hkv, g.NHG, g.D, g.dtype, g.NW, pws,
+                    g.lay.prefix, g.lay.wplan, g.lay.counters};
+  };
+  plan2_kernel<<<2, kPlanThreads, 0, st>>>(
+      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws),
+      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws));
+  rc = host::check_launch();
   if (rc != PKV_OK) return rc;
-  rc = run_impl(w + c.q_grp, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.grp_table),
-                max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
-                num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
-                w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, false, 0,
-                reinterpret_cast<float*>(w + c.lse_p));
-  if (rc != PKV_OK) return rc;
-  // suffix pass: each request over its own blocks
-  rc = do_plan(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws, st);
-  if (rc != PKV_OK) return rc;
+  // own-part pass: each request over its own blocks
   rc = run_impl(q, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.suf_table), max_blocks_per_seq,
                 reinterpret_cast<const int32_t*>(w + c.suf_len), num_seqs, num_q_heads, num_kv_heads, head_dim,
                 block_size, num_blocks, scale, kv_dtype, w + c.o_s, PKV_F32, w + c.suf_ws, c.gs.lay.total,
                 stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
+  if (rc != PKV_OK) return rc;
+  // shared-part pass: groups x members, every member sees the whole shared
+  // part.  It may start during the own-part pass's tail (launch overlap):
+  // what it reads first -- its plan, the group tables and lengths, the pools
+  // -- was written by the gather and plan kernels, which finished before
+  // the own-part pass began; that pass writes only its own workspace and o_s.
+  rc = run_impl(w + c.q_grp, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.grp_table),
+                max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
+                num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
+                w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, true, 0,
+                reinterpret_cast<float*>(w + c.lse_p));
   if (rc != PKV_OK) return rc;
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
   const int threads = 256;
