@@ -65,7 +65,7 @@ def parse():
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
     p.add_argument("--no-extras", action="store_true", help="skip the measurements of the other rows")
     p.add_argument("--extra", default=None,
-                   choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving"],
+                   choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving", "mixed_512"],
                    help="run only this one extra measurement and print its JSON (for profiling captures)")
     p.add_argument("--no-overlap", action="store_true",
                    help="launch every layer's attention without programmatic dependent launch")
@@ -455,12 +455,29 @@ def cpu_baseline(seconds: float):
             if compute >= seconds:
                 break
         layers += 1
+    # the two small batches, whole (one layer each)
+    others = {}
+    for name in ("tiny", "mixed_512"):
+        wo = W.workload(name)
+        go = W.rng(wo.seed + 100)
+        tot = 0.0
+        nbytes = 0
+        for n in wo.lengths:
+            kh, vh = W.kv_history(go, wo, n), W.kv_history(go, wo, n)
+            q = (W.normal_bf16_bits if wo.dtype == "bf16" else W.normal_f32)(go, (wo.num_q_heads, wo.head_dim))
+            t1 = time.perf_counter()
+            oatt.dense_decode(q, kh, vh, wo.scale)
+            tot += time.perf_counter() - t1
+            es = 2 if wo.dtype == "bf16" else 4
+            nbytes += n * wo.num_kv_heads * wo.head_dim * es * 2 + 2 * wo.num_q_heads * wo.head_dim * es
+        others[name] = {"seconds": tot, "gb_per_s": nbytes / tot / 1e9, "requests": len(wo.lengths)}
     return {"value": done_bytes / compute / 1e9, "unit": "GB/s", "cores": _blas_threads(),
             "host_cpus": os.cpu_count(), "kind": "oracle",
             "sample": f"float64 NumPy dense decode attention of {n_att} (request, layer) pairs of the "
                       f"32 requests x 4096 history (H_q 32, H_kv 8, d 128; histories drawn once and "
                       f"reused across {layers} layers, fresh q per layer); {compute:.1f} s of CPU work, "
-                      f"input generation not timed"}
+                      f"input generation not timed",
+            "other_batches_one_layer": others}
 
 
 def swap_measurement():
@@ -658,6 +675,34 @@ def large_serving_measurement(reps: int = 12):
     return {"us_per_layer": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9, "kv_tokens": int(lens.sum())}
 
 
+def mixed_512_measurement(reps: int = 20):
+    """512 requests with lengths uniform in 1..512 (H_q 32, H_kv 8, d 128,
+    bf16, B 16): one layer of short ragged histories per call."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    import workloads as W
+
+    wl = W.workload("mixed_512", block_size=16)
+    S, Hq, Hkv, D, B, N = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.pool_blocks
+    a = pkv.BlockAllocator(N, B, free_order=W.free_order(W.rng(wl.seed), N))
+    for i, n in enumerate(wl.lengths):
+        assert a.add_seq(i, n) == 0
+    tables, lens = a.fill_tables(list(range(S)), -(-max(wl.lengths) // B))
+    td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    pools = [(torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16),
+              torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16)) for _ in range(4)]
+    q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
+    ws = pkv.new_workspace(S, Hq, Hkv, D)
+    us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
+    nbytes = (int(lens.sum()) * Hkv * D * 2 * 2 + 2 * S * Hq * D * 2
+              + 4 * int(sum(-(-int(n) // B) for n in lens)) + 4 * S)
+    del pools
+    return {"us_per_layer": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9, "kv_tokens": int(lens.sum())}
+
+
 def allocator_measurement(seconds: float = 1.0):
     """Host allocator throughput (C++): admit with prefix-cache hits, decode
     appends, release, on a 4096-block pool; operations per second."""
@@ -739,6 +784,7 @@ EXTRAS = {
     "multi_query": lambda: multi_query_measurement(),
     "prefix_cow": lambda: prefix_cow_measurement(),
     "large_serving": lambda: large_serving_measurement(),
+    "mixed_512": lambda: mixed_512_measurement(),
 }
 
 
@@ -811,7 +857,8 @@ def main():
             extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement(),
                       "multi_query_32x4096": multi_query_measurement(),
                       "prefix_cow_256x2264": prefix_cow_measurement(),
-                      "large_serving_256xU8192": large_serving_measurement()}
+                      "large_serving_256xU8192": large_serving_measurement(),
+                      "mixed_512xU512": mixed_512_measurement()}
         steps_per_s = args.steps / (ms_max / 1000) * world
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
