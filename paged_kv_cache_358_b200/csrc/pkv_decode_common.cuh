@@ -131,14 +131,14 @@ struct TileLim {
   int nvalid;  // rows holding tokens of the request (1..16)
   int rem;     // length - first position of the tile (may exceed 16)
   int T;       // query tokens per request
-  int Gq;      // grouped query heads per KV head
+  int gq_mul;  // ceil(2^16 / Gq): c / Gq == (c * gq_mul) >> 16 for every column c < 16
   int causal_on;  // 0: the T tokens all see the whole history (columns differ only in q)
   PKV_DEVINL int lim(int c) const {
     if constexpr (!kCausal) {
       return nvalid;
     } else {
       if (!causal_on) return nvalid;
-      const int causal_lim = rem - (T - 1 - c / Gq);
+      const int causal_lim = rem - (T - 1 - ((c * gq_mul) >> 16));
       return causal_lim < nvalid ? causal_lim : nvalid;
     }
   }

@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
   const int T = MULTI ? a.num_q_tokens : 1;
   const int Gq = MULTI ? Hq / Hkv : G;
   const int ncols = MULTI ? T * Gq : G;
+  const int gq_mul = ((1 << 16) + Gq - 1) / Gq;  // exact division of column indices < 16 by Gq
   const int box_rows = Bsz < kTile ? Bsz : kTile;
   const int nbox = kTile / box_rows;  // boxes per tile per chunk
   const uint64_t pol = policy_evict_first();
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       }
       __syncwarp();
     }
-    const TileLim<MULTI> lim{nvalid, MULTI ? m.len - m.j * kTile : nvalid, T, Gq, a.causal};
+    const TileLim<MULTI> lim{nvalid, MULTI ? m.len - m.j * kTile : nvalid, T, gq_mul, a.causal};
     if constexpr (Core::kSwizzle) {
       Core::tile(state, stage + Core::kKOff, stage + Core::kVOff, lim, a.scale_log2, lane);
     } else {
