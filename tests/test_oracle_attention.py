@@ -253,3 +253,87 @@ def test_multi_query_special_cases():
     clean = att.multi_query(q, K, V, 0.25)
     assert np.array_equal(pois[:2], clean[:2])      # tokens at positions 2, 3
     assert np.isnan(pois[2:]).all()
+
+
+# -- per-head checker and the bf16 decoder -------------------------------------
+# ``dense_decode_head`` is the checker of the full-size sampled parity tests and
+# ``widen`` decodes every bf16 bit pattern on the oracle's side; both are pinned
+# here against library routines and exact values, not against other oracle code.
+def _sdpa_head_f64(q_h, K, V, scale):
+    """q_h [d], K/V [n, d] float64 -> [d] via torch SDPA (one head)."""
+    qt = torch.from_numpy(np.ascontiguousarray(q_h))[None, None, None, :]
+    kt = torch.from_numpy(np.ascontiguousarray(K))[None, None]
+    vt = torch.from_numpy(np.ascontiguousarray(V))[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+    return out[0, 0, 0].numpy()
+
+
+def _bf16_bits_to_f64_torch(bits):
+    """bf16 bit patterns -> float64 through torch's own bfloat16 conversion on the CPU."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("n,H_q,H_kv,d,kind,qscale",
+                         [(1, 4, 1, 8, "f32", 1.0), (5, 8, 2, 16, "f32", 1.0), (37, 8, 2, 64, "bf16", 1.0),
+                          (200, 32, 8, 128, "bf16", 1.0), (64, 32, 4, 128, "bf16", 1000.0),
+                          (17, 16, 4, 32, "f32", 1000.0), (300, 8, 8, 128, "bf16", 30.0)])
+def test_dense_decode_head_matches_sdpa(n, H_q, H_kv, d, kind, qscale):
+    """Every (query head h, KV head h // G) through the per-head checker equals
+    torch SDPA in float64 on the same widened values, for float32 and bf16 bit
+    inputs, with logits up to |s| ~ 1e3."""
+    g = rng(700 + n + d)
+    draw = normal_f32 if kind == "f32" else normal_bf16_bits
+    q = draw(g, (H_q, d), qscale)
+    K = draw(g, (n, H_kv, d))
+    V = draw(g, (n, H_kv, d))
+    scale = 1.0 / np.sqrt(d)
+    G = H_q // H_kv
+    qf = q.astype(np.float64) if kind == "f32" else _bf16_bits_to_f64_torch(q)
+    Kf = K.astype(np.float64) if kind == "f32" else _bf16_bits_to_f64_torch(K)
+    Vf = V.astype(np.float64) if kind == "f32" else _bf16_bits_to_f64_torch(V)
+    for h in range(H_q):
+        out = att.dense_decode_head(q[h], K[:, h // G], V[:, h // G], scale)
+        assert np.all(np.isfinite(out))
+        ref = _sdpa_head_f64(qf[h], Kf[:, h // G], Vf[:, h // G], scale)
+        assert np.max(np.abs(out - ref)) < 1e-12, (h, np.max(np.abs(out - ref)))
+
+
+def test_dense_decode_head_special_cases():
+    g = rng(71)
+    d = 32
+    # length 0 -> zeros of the head's width
+    z = att.dense_decode_head(normal_f32(g, (d,)), np.zeros((0, d), np.float32), np.zeros((0, d), np.float32), 0.5)
+    assert z.shape == (d,) and not z.any()
+    # length 1 -> v_0 exactly (bf16 input)
+    K1, V1 = normal_bf16_bits(g, (1, d)), normal_bf16_bits(g, (1, d))
+    one = att.dense_decode_head(normal_bf16_bits(g, (d,)), K1, V1, 0.25)
+    assert np.array_equal(one, _bf16_bits_to_f64_torch(V1)[0])
+    # one dominant logit selects that token's value
+    K = normal_f32(g, (40, d))
+    V = normal_f32(g, (40, d))
+    dom = att.dense_decode_head(K[23] * 1000.0, K, V, 1.0)
+    np.testing.assert_allclose(dom, V[23].astype(np.float64), rtol=0, atol=1e-12)
+
+
+def test_widen_matches_torch_bfloat16():
+    """The bf16 decoder against torch's bfloat16 -> float64 conversion over every
+    one of the 65,536 bit patterns (NaNs compared as NaN), and exact values."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):   # signalling-NaN patterns
+        ours = att.widen(bits)
+    ref = _bf16_bits_to_f64_torch(bits)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+    fixed = {0x3F80: 1.0, 0xC000: -2.0, 0x0000: 0.0, 0x4049: 3.140625, 0x3F00: 0.5,
+             0x0001: 2.0 ** -133, 0x0080: 2.0 ** -126, 0x7F7F: (2.0 - 2.0 ** -7) * 2.0 ** 127,
+             0x7F80: np.inf, 0xFF80: -np.inf}
+    for b, v in fixed.items():
+        assert att.widen(np.array([b], np.uint16))[0] == v, hex(b)
+    neg0 = att.widen(np.array([0x8000], np.uint16))[0]
+    assert neg0 == 0.0 and np.signbit(neg0)
+    # float inputs pass through exactly
+    x = normal_f32(rng(72), (100,))
+    assert np.array_equal(att.widen(x), x.astype(np.float64))

@@ -192,3 +192,46 @@ def test_unmutated_multi_query_passes_pins():
 def test_multi_query_mutant_is_caught(monkeypatch):
     monkeypatch.setattr(att, "multi_query", _multi_query_off_by_one)
     assert _any_pin_fails(MQ_PINS)
+
+
+# -- per-head checker and bf16 decoder mutants ---------------------------------
+def _head_no_max_shift(q_h, k_head, v_head, scale):
+    qh, K, V = att.widen(q_h), att.widen(k_head), att.widen(v_head)
+    if K.shape[0] == 0:
+        return np.zeros(qh.shape[0])
+    e = np.exp(float(scale) * (K @ qh))     # overflows at |s| ~ 1e3
+    return (e / e.sum()) @ V
+
+
+def _head_scale_squared(q_h, k_head, v_head, scale):
+    return att.__dict__["_orig_head"](q_h, k_head, v_head, float(scale) ** 2)
+
+
+def _widen_shift_15(x):
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
+HEAD_PINS = [lambda: TA.test_dense_decode_head_matches_sdpa(64, 32, 4, 128, "bf16", 1000.0),
+             lambda: TA.test_dense_decode_head_matches_sdpa(5, 8, 2, 16, "f32", 1.0),
+             TA.test_dense_decode_head_special_cases]
+WIDEN_PINS = [TA.test_widen_matches_torch_bfloat16]
+
+
+def test_unmutated_head_and_widen_pass_pins():
+    assert not _any_pin_fails(HEAD_PINS)
+    assert not _any_pin_fails(WIDEN_PINS)
+
+
+@pytest.mark.parametrize("mutant", [_head_no_max_shift, _head_scale_squared])
+def test_head_mutants_are_caught(monkeypatch, mutant):
+    monkeypatch.setitem(att.__dict__, "_orig_head", att.dense_decode_head)
+    monkeypatch.setattr(att, "dense_decode_head", mutant)
+    assert _any_pin_fails(HEAD_PINS)
+
+
+def test_widen_mutant_is_caught(monkeypatch):
+    monkeypatch.setattr(att, "widen", _widen_shift_15)
+    assert _any_pin_fails(WIDEN_PINS)
