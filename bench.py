@@ -65,12 +65,15 @@ def parse():
     p.add_argument("--kernel", type=int, default=0, help="0 auto, 1 FMA tiles, 2 tensor-core tiles")
     p.add_argument("--no-extras", action="store_true", help="skip the measurements of the other rows")
     p.add_argument("--extra", default=None,
-                   choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving", "mixed_512"],
+                   choices=["swap", "allocator", "multi_query", "prefix_cow", "large_serving", "mixed_512",
+                            "large_serving_steps", "prefix_cow_steps", "block_size_sweep", "hbm_ceiling"],
                    help="run only this one extra measurement and print its JSON (for profiling captures)")
     p.add_argument("--no-overlap", action="store_true",
                    help="launch every layer's attention without programmatic dependent launch")
     p.add_argument("--unfused", action="store_true",
                    help="append with a separate kv_append launch instead of folding it into attention")
+    p.add_argument("--pool-copies", type=int, default=None,
+                   help="pool copies the multi_query extra rotates over (fewer: smaller profiling captures)")
     p.add_argument("--layers", type=int, default=32,
                    help="layers per step (32 for the workload; fewer only for small profiling captures)")
     return p.parse_args()
@@ -201,35 +204,63 @@ class ClockSampler:
 
 # -- the workload -------------------------------------------------------------------
 class DecodeStep:
-    """32-layer decode step through the C ABI; all state resident on the device."""
+    """Multi-layer decode step through the C ABI; all state resident on the device.
+
+    workload: a name of ``workloads.workload`` (its lengths, heads, head_dim,
+    block size).  prefix_groups = (groups, branches, prompt): instead of the
+    workload's lengths, `groups` prompts of `prompt` tokens are admitted and
+    each is forked to `branches` requests that share its blocks (copy-on-write
+    of the shared partial tail on the first append).  shared_prefix: attend
+    through the shared-prefix call (each group's shared blocks read once per
+    layer) after a separate kv_append, instead of the folded append."""
 
     def __init__(self, steps_budget: int, seed: int, kernel: int, rank: int = 0, world: int = 1,
-                 layers: int = 32, fused: bool = True, overlap: bool = True):
+                 layers: int = 32, fused: bool = True, overlap: bool = True,
+                 workload: str = "teaching_32x4096", prefix_groups=None, shared_prefix: bool = False):
         import torch
 
         import paged_kv_cache_358_b200 as pkv
         import workloads as W
 
         self.torch, self.pkv = torch, pkv
-        self.fused = fused
+        self.fused = fused and not shared_prefix
+        self.shared_prefix = shared_prefix
         # layers after the first may start while the previous layer's launch
         # finishes (each reads its own pool; the plan, tables and slots were
         # written by kernels that completed before layer 0 started)
         self.overlap = overlap
         pkv.set_decode_kernel(kernel)
-        wl = W.workload("teaching_32x4096", decode_steps=steps_budget + 8, seed=seed)
+        wl = W.workload(workload, decode_steps=steps_budget + 8, seed=seed)
         self.wl = wl
-        S, L, Hq, Hkv, D, B = wl.num_seqs, layers, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+        Hq, Hkv, D, B = wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+        if prefix_groups is not None:
+            ng, br, prompt = prefix_groups
+            lengths = [prompt] * (ng * br)
+            # prompts (full blocks + tail) + per request its copied tail and appends
+            N = ng * -(-prompt // B) + ng * br * (-(-(B + steps_budget + 8) // B) + 1)
+        else:
+            lengths = list(wl.lengths)
+            N = wl.pool_blocks
+        S, L = len(lengths), layers
         self.S, self.L, self.Hq, self.Hkv, self.D, self.B = S, L, Hq, Hkv, D, B
-        N = wl.pool_blocks
         self.N = N
         g = W.rng(seed)
         order = W.free_order(g, N)
         self.alloc = pkv.BlockAllocator(N, B, free_order=order)
         self.ids = np.array(list(shard_requests(S, world, rank)), dtype=np.int32)
-        for i, n in zip(self.ids, wl.lengths):
-            assert self.alloc.add_seq(int(i), n) == 0
-        self.max_blocks = -(-(max(wl.lengths) + steps_budget + 8) // B)
+        if prefix_groups is not None:
+            for gi in range(ng):
+                root = int(self.ids[gi * br])
+                assert self.alloc.add_seq(root, prompt) == 0
+                for b in range(1, br):
+                    assert self.alloc.fork(root, int(self.ids[gi * br + b])) == 0
+            self.group_start = torch.arange(0, S + 1, br, dtype=torch.int32, device="cuda")
+            self.prefix_blocks = torch.full((ng,), prompt // B, dtype=torch.int32, device="cuda")
+            self.max_group = br
+        else:
+            for i, n in zip(self.ids, lengths):
+                assert self.alloc.add_seq(int(i), n) == 0
+        self.max_blocks = -(-(max(lengths) + steps_budget + 8) // B)
         dev = torch.device("cuda")
         gen = torch.Generator(device=dev)
         gen.manual_seed(seed)
@@ -263,6 +294,9 @@ class DecodeStep:
         self.cp_d = torch.empty((S, 3), dtype=torch.int32, device=dev)
         self.slots = torch.empty((S,), dtype=torch.int64, device=dev)
         self.ws = pkv.new_workspace(S, Hq, Hkv, D)
+        if shared_prefix:
+            self.wsp = pkv.shared_prefix_workspace(S, len(self.prefix_blocks), self.max_group, Hq, Hkv, D,
+                                                   self.max_blocks)
         self.stream = torch.cuda.current_stream()
         self.parity = 0
         self.launches = 0
@@ -270,6 +304,7 @@ class DecodeStep:
         self.attn_bytes = []
         self.attn_events = []
         self.record_attn = False
+        self.step_events = None    # when a list: one event recorded at the end of each step
         # e2e host buffers and copy streams: step k's inputs go up on one stream
         # (while step k-1 computes) and its outputs come back on another (while
         # step k+1 computes); events order every copy against the kernels
@@ -283,14 +318,16 @@ class DecodeStep:
         self.step_done = [None, None]   # per buffer: its step's kernels finished
         self.out_back = [None, None]    # per buffer: its step's outputs on the host
 
-    def bytes_of_step(self, lens: np.ndarray, n_copies: int) -> int:
-        """Algorithmic bytes: every history slot read once per KV head, q, out, appends, metadata."""
+    def bytes_of_step(self, lens: np.ndarray, copied_rows: int) -> int:
+        """Algorithmic bytes: every history slot read once per KV head, q, out, appends,
+        metadata, and the copy-on-write copies (`copied_rows` = the sum of n_valid
+        over the step's copies: only the valid slots of a shared tail are copied)."""
         e = 2
         kv = int(lens.sum()) * self.Hkv * self.D * e * 2
         qo = self.S * self.Hq * self.D * e * 2
         app = self.S * self.Hkv * self.D * e * 2 * 2
         meta = 4 * int(sum(-(-int(n) // self.B) for n in lens)) + 4 * self.S
-        cow = n_copies * self.B * self.Hkv * self.D * e * 2 * 2
+        cow = copied_rows * self.Hkv * self.D * e * 2 * 2
         return self.L * (kv + qo + app + meta) + self.L * cow + 8 * self.S
 
     def attn_bytes_per_launch(self, lens: np.ndarray) -> int:
@@ -330,8 +367,10 @@ class DecodeStep:
             pkv.block_copy(self.k_pools, self.v_pools, self.cp_d[:nc])
             self.launches += 1
         pkv.slot_mapping(self.tab_d, self.pos_d, self.B, out=self.slots)
-        pkv.decode_plan(self.len_d, self.Hq, self.Hkv, self.D, pkv.BF16, self.ws)
-        self.launches += 2
+        self.launches += 1
+        if not self.shared_prefix:      # the shared-prefix call plans inside each layer's call
+            pkv.decode_plan(self.len_d, self.Hq, self.Hkv, self.D, pkv.BF16, self.ws)
+            self.launches += 1
         eb = 0
         if e2e:
             eb = self.e2e_k % 2
@@ -358,6 +397,14 @@ class DecodeStep:
             if not self.fused:
                 pkv.kv_append(k_new[i], v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
                 self.launches += 1
+            if self.shared_prefix:
+                # memset + gather + both plans + two attention passes + combine
+                pkv.paged_decode_attn_shared_prefix(q[i], self.k_pools[i], self.v_pools[i], self.tab_d,
+                                                    self.len_d, self.group_start, self.prefix_blocks,
+                                                    self.max_group, self.wl.scale, out=out[i],
+                                                    workspace=self.wsp)
+                self.launches += 5
+                continue
             pkv.set_launch_overlap(self.overlap and i > 0 and self.fused)
             if self.fused:
                 pkv.paged_decode_attn_append_run(q[i], k_new[i], v_new[i], self.slots,
@@ -381,7 +428,11 @@ class DecodeStep:
             e1.record(self.stream)
             self.attn_events.append((e0, e1))
             self.attn_bytes.append(self.attn_bytes_per_launch(lens))
-        self.bytes_done += self.bytes_of_step(lens, nc)
+        self.bytes_done += self.bytes_of_step(lens, int(self.copies_h[:nc, 2].sum()) if nc else 0)
+        if self.step_events is not None:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record(self.stream)
+            self.step_events.append(ev)
 
     def drain(self):
         """Order the compute stream after the last outputs' copy to the host."""
@@ -396,7 +447,7 @@ class DecodeStep:
         return self.L * per_layer_in + meta, self.L * self.S * self.Hq * self.D * e
 
 
-def timed(fn, steps, dist, stream, finish=None):
+def timed(fn, steps, dist, stream, finish=None, start=None):
     import torch
 
     if dist is not None:
@@ -405,6 +456,8 @@ def timed(fn, steps, dist, stream, finish=None):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.perf_counter()
     e0.record(stream)
+    if start is not None:
+        start()
     for _ in range(steps):
         fn()
     if finish is not None:
@@ -416,6 +469,14 @@ def timed(fn, steps, dist, stream, finish=None):
         dist.barrier()
     ms = e0.elapsed_time(e1)
     return ms, wall
+
+
+def step_stats(step_ms) -> dict:
+    """Median, 10th and 90th percentile and mean of per-step device times (ms),
+    from one CUDA event recorded at the end of every timed step."""
+    x = np.asarray(step_ms, dtype=np.float64)
+    return {"median": float(np.median(x)), "p10": float(np.percentile(x, 10)),
+            "p90": float(np.percentile(x, 90)), "mean": float(x.mean()), "n": int(x.size)}
 
 
 # -- CPU oracle baseline -----------------------------------------------------------
@@ -509,7 +570,7 @@ def swap_measurement():
     return res
 
 
-def multi_query_measurement(reps: int = 20):
+def multi_query_measurement(reps: int = 20, copies: int = 12):
     """Multi-token query (T tokens per request, causal) on one layer of the
     32 x 4096 teaching shapes: microseconds per call (plan + attention) and
     algorithmic GB/s (history K/V once per KV head, q and out of all T tokens,
@@ -529,7 +590,6 @@ def multi_query_measurement(reps: int = 20):
     td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
-    copies = 12
     kp = [torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
     vp = [torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
     res = {}
@@ -539,7 +599,7 @@ def multi_query_measurement(reps: int = 20):
         ws = torch.zeros(pkv.lib().pkv_multi_query_workspace_bytes(S, T, Hq, Hkv, D), dtype=torch.uint8,
                          device="cuda")
         for i in range(3):
-            pkv.paged_attn_multi_query(q, kp[i], vp[i], td, ld, wl.scale, out=out, workspace=ws)
+            pkv.paged_attn_multi_query(q, kp[i % copies], vp[i % copies], td, ld, wl.scale, out=out, workspace=ws)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -703,6 +763,127 @@ def mixed_512_measurement(reps: int = 20):
     return {"us_per_layer": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9, "kv_tokens": int(lens.sum())}
 
 
+def serving_steps_measurement(kind: str, steps: int, layers: int = 24, shared_prefix: bool = False):
+    """Whole decode steps of a serving batch, timed with one CUDA event per step.
+
+    kind "large_serving": 256 requests, lengths U(1..8192), H_q 32 / H_kv 4
+    (G = 8), d 128, bf16, B 16, 24 layers; every step appends one token per
+    request (allocator, table mirror, slot mapping, plan, then one launch per
+    layer with the append folded in).
+    kind "prefix_cow": 64 prompts of 2008 tokens, each forked to 4 branches
+    (H_q 16 / H_kv 4, d 128, bf16, B 16, 24 layers); the timed steps start at
+    the first append, so the copy-on-write of every shared 8-token tail (3 per
+    group, in all 24 layers) is inside the timed region.  With shared_prefix
+    each layer runs kv_append and the shared-prefix call (each group's 125
+    shared blocks read once) instead of the folded append.
+    Reports ms per step (median and mean), steps/s, tokens/s and the
+    algorithmic GB/s of the step (every request's history counted: logical);
+    for prefix_cow also GB/s of the unique blocks of the pool."""
+    import torch
+
+    if kind == "prefix_cow":
+        ds = DecodeStep(steps + 8, 3, 0, layers=layers, workload="prefix_cow", prefix_groups=(64, 4, 2008),
+                        shared_prefix=shared_prefix)
+        warm = 0        # the first append (copy-on-write) is timed; the kernels are warm already
+    else:
+        ds = DecodeStep(steps + 8, 4, 0, layers=layers, workload="large_serving")
+        warm = 3
+    for _ in range(warm):
+        ds.step()
+    torch.cuda.synchronize()
+    ds.bytes_done = 0
+    copies0 = ds.alloc.stats()["cow_copies"]
+    start_ev = torch.cuda.Event(enable_timing=True)
+    ds.step_events = []
+    ms, _ = timed(ds.step, steps, None, ds.stream, start=lambda: start_ev.record(ds.stream))
+    marks = [start_ev] + ds.step_events
+    step_ms = np.array([a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])])
+    assert ds.pkv.decode_status(ds.wsp if shared_prefix else ds.ws) == 0
+    st = ds.alloc.stats()
+    res = {"layers": layers, "requests": ds.S, "steps": steps, "ms_per_step": ms / steps,
+           "step_ms": step_stats(step_ms), "steps_per_s": steps / (ms / 1000),
+           "tokens_per_s": steps * ds.S / (ms / 1000), "gb_per_s": ds.bytes_done / (ms / 1000) / 1e9,
+           "kv_tokens_end": int(sum(ds.alloc.length(int(i)) for i in ds.ids)),
+           "cow_copies": int(st["cow_copies"] - copies0)}
+    if kind == "prefix_cow":
+        # unique bytes: each physical block of the pool read once per layer (upper bound: whole blocks)
+        row = ds.Hkv * ds.D * 2 * 2
+        res["unique_blocks_end"] = int(st["active"])
+        res["unique_gb_per_s_upper"] = (steps * layers * st["active"] * ds.B * row) / (ms / 1000) / 1e9
+    del ds
+    torch.cuda.empty_cache()
+    return res
+
+
+def block_size_sweep_measurement(reps: int = 20):
+    """The 512 short ragged requests (lengths U{1..512}, H_q 32 / H_kv 8, d 128,
+    bf16) at block sizes 4, 8, 16, 32, 64: microseconds per layer (plan +
+    attention), algorithmic GB/s, and the mean tail waste (slots allocated
+    past the length, B * ceil(n / B) - n) beside its expectation (B - 1) / 2."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+    import workloads as W
+
+    res = {}
+    for B in (4, 8, 16, 32, 64):
+        wl = W.workload("mixed_512", block_size=B)
+        S, Hq, Hkv, D, N = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.pool_blocks
+        a = pkv.BlockAllocator(N, B, free_order=W.free_order(W.rng(wl.seed), N))
+        for i, n in enumerate(wl.lengths):
+            assert a.add_seq(i, n) == 0
+        tables, lens = a.fill_tables(list(range(S)), -(-max(wl.lengths) // B))
+        td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(11 + B)
+        pools = [(torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16),
+                  torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16))
+                 for _ in range(4)]
+        q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
+        ws = pkv.new_workspace(S, Hq, Hkv, D)
+        us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
+        nbytes = (int(lens.sum()) * Hkv * D * 2 * 2 + 2 * S * Hq * D * 2
+                  + 4 * int(sum(-(-int(n) // B) for n in lens)) + 4 * S)
+        waste = [B * -(-int(n) // B) - int(n) for n in lens]
+        res[f"B{B}"] = {"us_per_layer": us, "gb_per_s": nbytes / (us * 1e-6) / 1e9,
+                        "mean_tail_waste_slots": float(np.mean(waste)), "expected_waste": (B - 1) / 2,
+                        "blocks": int(sum(-(-int(n) // B) for n in lens))}
+        del pools
+    return res
+
+
+def hbm_ceiling_measurement(reps: int = 10):
+    """Context for the roofline: what plain library kernels stream on this GPU.
+    A read-only reduction (torch amax over 4 GiB of int32) and a copy (2 GiB
+    read + 2 GiB written), each timed with CUDA events over `reps` calls, in
+    GB/s of bytes moved.  The decode kernel only reads (its writes are < 1 %),
+    so the read-only figure is its practical ceiling."""
+    import torch
+
+    n = (4 << 30) // 4
+    x = torch.randint(0, 1 << 30, (n,), dtype=torch.int32, device="cuda")
+    res = {}
+    for name, fn, nbytes in (("read_only_amax", lambda: torch.amax(x), 4 << 30),
+                             ("copy", None, 4 << 30)):
+        if fn is None:
+            src, dst = x[: n // 2], x[n // 2:]
+            fn = lambda: dst.copy_(src)
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms": ms, "gb_per_s": nbytes / (ms * 1e-3) / 1e9}
+    del x
+    torch.cuda.empty_cache()
+    return res
+
+
 def allocator_measurement(seconds: float = 1.0):
     """Host allocator throughput (C++): admit with prefix-cache hits, decode
     appends, release, on a 4096-block pool; operations per second."""
@@ -785,6 +966,12 @@ EXTRAS = {
     "prefix_cow": lambda: prefix_cow_measurement(),
     "large_serving": lambda: large_serving_measurement(),
     "mixed_512": lambda: mixed_512_measurement(),
+    "large_serving_steps": lambda: serving_steps_measurement("large_serving", 64),
+    "prefix_cow_steps": lambda: {"plain": serving_steps_measurement("prefix_cow", 256),
+                                 "shared_prefix": serving_steps_measurement("prefix_cow", 256,
+                                                                            shared_prefix=True)},
+    "block_size_sweep": lambda: block_size_sweep_measurement(),
+    "hbm_ceiling": lambda: hbm_ceiling_measurement(),
 }
 
 
@@ -794,7 +981,11 @@ def main():
         reference_arm(args)
         return
     if args.extra is not None:
-        print(json.dumps({args.extra: EXTRAS[args.extra]()}), flush=True)
+        if args.extra == "multi_query" and args.pool_copies:
+            res = multi_query_measurement(copies=args.pool_copies)
+        else:
+            res = EXTRAS[args.extra]()
+        print(json.dumps({args.extra: res}), flush=True)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
     import torch
@@ -820,8 +1011,17 @@ def main():
     ds.bytes_done = 0
     ds.launches = 0
     ds.record_attn = True
-    ms, wall = timed(ds.step, args.steps, dist, stream)
+    start_ev = torch.cuda.Event(enable_timing=True)
+    ds.step_events = []
+
+    def first_event():
+        start_ev.record(stream)
+
+    ms, wall = timed(ds.step, args.steps, dist, stream, start=first_event)
     ds.record_attn = False
+    marks = [start_ev] + ds.step_events
+    step_ms = np.array([a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])])
+    ds.step_events = None
     clk = clocks.stop()
     launches = ds.launches
     step_bytes = ds.bytes_done
@@ -854,11 +1054,20 @@ def main():
             cpu = cpu_baseline(args.cpu_seconds)
         extras = None
         if world == 1 and not args.no_extras:
+            # the headline batch's pools are not needed any more
+            ds.k_pools = ds.v_pools = None
+            torch.cuda.empty_cache()
             extras = {"swap_500mib": swap_measurement(), "allocator": allocator_measurement(),
                       "multi_query_32x4096": multi_query_measurement(),
                       "prefix_cow_256x2264": prefix_cow_measurement(),
                       "large_serving_256xU8192": large_serving_measurement(),
-                      "mixed_512xU512": mixed_512_measurement()}
+                      "mixed_512xU512": mixed_512_measurement(),
+                      "large_serving_steps_24L": serving_steps_measurement("large_serving", 64),
+                      "prefix_cow_steps_24L": {
+                          "plain": serving_steps_measurement("prefix_cow", 256),
+                          "shared_prefix": serving_steps_measurement("prefix_cow", 256, shared_prefix=True)},
+                      "mixed_512_block_size_sweep": block_size_sweep_measurement(),
+                      "hbm_ceiling_4gib": hbm_ceiling_measurement()}
         steps_per_s = args.steps / (ms_max / 1000) * world
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -872,6 +1081,7 @@ def main():
                        "parallelism": f"replicas x{world} (requests sharded by rank, no collective)",
                        "launch_overlap": bool(ds.overlap and ds.fused)},
             "steps_per_s": steps_per_s, "tokens_per_s": steps_per_s * ds.S,
+            "step_ms": step_stats(step_ms),
             "frac_of_nominal_8tbs": value / NOMINAL_HBM_GBS,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e_max / args.steps},

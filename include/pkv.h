@@ -176,7 +176,8 @@ int pkv_paged_decode_attn_append_run(const void* q, const void* k_new, const voi
  * Arguments are those of pkv_paged_decode_attn without the workspace.
  * - Batches whose pkv_decode_workspace_bytes() exceeds 16 MiB are refused
  *   with PKV_ERR_INVALID (pkv_last_cuda_error() says why); nothing runs.
- * - The first call on each device looks up the array's device address; make
+ * - The first call on each device (and the first after a cudaDeviceReset,
+ *   which creates a new context) looks up the array's device address; make
  *   that first call before any stream capture.
  * - No call allocates: no cudaMalloc/cudaFree, no allocating library routine.
  * - All calls share the one array per device: calls that overlap on the GPU
@@ -246,8 +247,10 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  *                 meaningful)
  * Other arguments as pkv_paged_decode_attn.  Five launches: a gather, both
  * plans, the own-part pass, the shared-part pass (the members' queries are
- * the columns of one launch; it starts during the own-part pass's tail), and
- * the combine. */
+ * the columns of one launch), and the combine.  The two passes run side by
+ * side: the plans split the SMs' worker slots between them in proportion to
+ * their tiles, and the shared-part pass, which reads nothing the own-part
+ * pass writes, starts without waiting for it. */
 size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_blocks_per_seq);

@@ -32,11 +32,45 @@ struct PlanArgs {
   int S, Hq, Hkv, NHG, D, kv_dtype, NW;
   char* ws;
   size_t off_prefix, off_wplan, off_counters;
+  int cost;  // relative cost of one of this plan's tiles (two plans sharing the SMs)
 };
 
+// Workers of the first of two launches that run side by side and share the
+// NW worker slots: proportional to the launches' costs (tiles x cost per
+// tile), at least one each when both have work.
+__device__ __forceinline__ int split_workers(long long tiles0, int cost0, long long tiles1, int cost1, int NW) {
+  const long long w0 = tiles0 * cost0, w1 = tiles1 * cost1;
+  if (w1 == 0) return NW;
+  if (w0 == 0) return 0;
+  long long n0 = (w0 * NW + (w0 + w1) / 2) / (w0 + w1);
+  if (n0 < 1) n0 = 1;
+  if (n0 > NW - 1) n0 = NW - 1;
+  return static_cast<int>(n0);
+}
+
+// Tiles of a request-length array (block reduction over one CTA), times NHG.
+__device__ long long block_total_tiles(const int32_t* __restrict__ seq_lens, int S, int NHG) {
+  __shared__ long long part[kPlanThreads / 32];
+  long long x = 0;
+  for (int s = threadIdx.x; s < S; s += kPlanThreads) x += ntiles_of(seq_lens[s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = x;
+  __syncthreads();
+  long long t = 0;
+  for (int w = 0; w < kPlanThreads / 32; ++w) t += part[w];
+  __syncthreads();
+  return t * NHG;
+}
+
+// NWa: the tiles are split over workers 0 .. NWa-1 (NWa <= NW, or a negative
+// value: compute it from `other`, a second plan whose launch runs side by side
+// with this one; `first` says which of the two this is).
 __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int S, int Hq, int Hkv,
                                           int NHG, int D, int kv_dtype, int NW, char* ws, size_t off_prefix,
-                                          size_t off_wplan, size_t off_counters) {
+                                          size_t off_wplan, size_t off_counters, int NWa = -1,
+                                          const PlanArgs* self = nullptr, const PlanArgs* other = nullptr,
+                                          bool first = true) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + off_prefix);
   int4* wplan = reinterpret_cast<int4*>(ws + off_wplan);
@@ -88,17 +122,25 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   __syncthreads();
   const long long T = total_seq_tiles * NHG;
   const int32_t* P = in_smem ? sp : prefix;
+  if (other != nullptr) {
+    const long long To = block_total_tiles(other->seq_lens, other->S, other->NHG);
+    const int n_first = first ? split_workers(T, self->cost, To, other->cost, NW)
+                              : split_workers(To, other->cost, T, self->cost, NW);
+    NWa = first ? n_first : NW - n_first;
+  }
+  if (NWa < 1 || NWa > NW) NWa = NWa < 1 ? 1 : NW;
 
-  // Worker v owns tiles [floor(v T / NW), floor((v+1) T / NW)); its first
-  // request is the last s with NHG * P[s] <= start (skipping empty requests).
+  // Worker v < NWa owns tiles [floor(v T / NWa), floor((v+1) T / NWa)); its
+  // first request is the last s with NHG * P[s] <= start (skipping empty
+  // requests).  Workers NWa .. NW-1 own none.
   for (int v = tid; v < NW; v += kPlanThreads) {
-    if (T == 0) {
+    if (T == 0 || v >= NWa) {
       wplan[2 * v] = make_int4(0, 0, 0, 0);
       wplan[2 * v + 1] = make_int4(0, 0, 0, 0);
       continue;
     }
-    const long long a = range_begin(v, T, NW);
-    const long long b = range_begin(v + 1, T, NW);
+    const long long a = range_begin(v, T, NWa);
+    const long long b = range_begin(v + 1, T, NWa);
     int lo = 0, hi = S - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -115,6 +157,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
     hdr->head_dim = D;
     hdr->kv_dtype = kv_dtype;
     hdr->num_workers = NW;
+    hdr->active_workers = NWa;
     hdr->head_groups = NHG;
     hdr->total_tiles = T;
     hdr->planned = 1;
@@ -126,14 +169,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int kv_dtype, int NW, char* ws,
                                                             size_t off_prefix, size_t off_wplan,
                                                             size_t off_counters) {
-  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters);
+  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters, NW);
 }
 
-// Two independent plans in one launch, one per CTA.
+// The plans of two launches that run side by side, one per CTA: the two
+// launches split the worker slots in proportion to their costs.
 __global__ void __launch_bounds__(kPlanThreads) plan2_kernel(const PlanArgs p0, const PlanArgs p1) {
-  const PlanArgs& p = blockIdx.x == 0 ? p0 : p1;
+  const bool first = blockIdx.x == 0;
+  const PlanArgs& p = first ? p0 : p1;
   plan_body(p.seq_lens, p.S, p.Hq, p.Hkv, p.NHG, p.D, p.kv_dtype, p.NW, p.ws, p.off_prefix, p.off_wplan,
-            p.off_counters);
+            p.off_counters, -1, &p, first ? &p1 : &p0, first);
 }
 
 }  // namespace pkv
@@ -317,7 +362,8 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
-             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr) {
+             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr,
+             int32_t independent = 0) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -358,6 +404,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.num_q_tokens = num_q_tokens;
   args.causal = causal;
   args.lse = lse;
+  args.independent = independent;
   geo.overlap = overlap;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
@@ -636,8 +683,12 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(workspace);
   const int32_t row_bytes = num_q_heads * head_dim * (kv_dtype == PKV_BF16 ? 2 : 4);
-  // The suffix workspace leads: clear its status word, the call's own.
+  // The suffix workspace leads: its status word is the call's own.  The
+  // shared-part pass records faults in its own sub-workspace, whose word the
+  // combine kernel folds into the call's; clear both, so a fault of an earlier
+  // call (or an uninitialised workspace) is never reported again.
   cudaError_t e = cudaMemsetAsync(w + c.suf_ws, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w + c.pre_ws, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return host::cuda_fail(e);
   cascade_gather_kernel<<<num_seqs, 128, 0, st>>>(
       static_cast<const char*>(q), block_tables, max_blocks_per_seq, seq_lens, num_seqs, group_start,
@@ -648,13 +699,16 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
   // both plans in one launch
-  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws) {
+  // The two passes run side by side and share the worker slots in
+  // proportion to their tiles, a shared-part tile (16 columns) costing about
+  // 1.35 times an own-part tile (the grouped heads of one query).
+  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws, int cost) {
     return PlanArgs{lens, g.S, g.Hq, g.Hkv, g.NHG, g.D, g.dtype, g.NW, pws,
-                    g.lay.prefix, g.lay.wplan, g.lay.counters};
+                    g.lay.prefix, g.lay.wplan, g.lay.counters, cost};
   };
   plan2_kernel<<<2, kPlanThreads, 0, st>>>(
-      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws),
-      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws));
+      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws, 20),
+      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws, 27));
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
   // own-part pass: each request over its own blocks
@@ -664,15 +718,19 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                 stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
   if (rc != PKV_OK) return rc;
   // shared-part pass: groups x members, every member sees the whole shared
-  // part.  It may start during the own-part pass's tail (launch overlap):
-  // what it reads first -- its plan, the group tables and lengths, the pools
-  // -- was written by the gather and plan kernels, which finished before
-  // the own-part pass began; that pass writes only its own workspace and o_s.
+  // part.  It runs side by side with the own-part pass (a programmatic
+  // dependent launch that never waits for it, on the worker slots the own-part
+  // plan leaves idle): everything it reads -- its plan, the grouped queries,
+  // the group tables and lengths, the pools -- was written by the gather and
+  // plan kernels, which finished before the own-part pass began, and it
+  // writes only its own workspace, o_p and lse_p, which the own-part pass
+  // does not touch.  Its one extra CTA waits for the own-part pass, so the
+  // combine kernel after it sees both results.
   rc = run_impl(w + c.q_grp, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.grp_table),
                 max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
                 num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
                 w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, true, 0,
-                reinterpret_cast<float*>(w + c.lse_p));
+                reinterpret_cast<float*>(w + c.lse_p), 1);
   if (rc != PKV_OK) return rc;
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
   const int threads = 256;
@@ -764,25 +822,62 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
+// The array's name is only a host-side stand-in in host code: its device
+// address is looked up with cudaGetSymbolAddress, with the device current,
+// once per device context and cached.  The cache is keyed by the context's
+// unique id, so after a cudaDeviceReset (a new context, the module loaded
+// again, possibly at another address) the first call looks the address up
+// again instead of using a stale one.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device.  The array's
-// name is only a host-side stand-in in host code, so the address is looked up
-// once per device (with that device current) and cached.
+struct NoAllocSlot {
+  unsigned long long ctx_id = 0;  // 0: not set up
+  void* ptr = nullptr;
+};
+
+std::mutex g_noalloc_mu;
+NoAllocSlot g_noalloc[64];
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return host::cuda_fail(e);
   if (dev < 0 || dev >= 64) return PKV_ERR_INVALID;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (!have_id || g_noalloc[dev].ctx_id != id) {
+    // set-up for this device context (also binds the context to the thread)
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return host::cuda_fail(e);
-    g_noalloc_ptr[dev] = p;
+    if (!have_id && !current_context_id(&id)) id = 0;  // no id: look the address up on every call
+    g_noalloc[dev].ctx_id = id;
+    g_noalloc[dev].ptr = p;
+    *out = p;
+    return PKV_OK;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = g_noalloc[dev].ptr;
   return PKV_OK;
 }
 
@@ -797,7 +892,9 @@ extern "C" int pkv_paged_decode_attn_noalloc(const void* q, const void* k_pool, 
                                              pkv_stream_t stream) {
   Geometry geo;
   if (!geometry(num_seqs, num_q_heads, num_kv_heads, head_dim, kv_dtype, &geo)) return PKV_ERR_INVALID;
-  if (geo.lay.total > kNoAllocScratchBytes) {
+  // the limit is the documented one: the workspace size pkv_decode_workspace_bytes
+  // states for the batch (the larger of the two storage types' layouts)
+  if (pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim) > kNoAllocScratchBytes) {
     host::set_error("decode batch needs more scratch than the 16 MiB built into the library");
     return PKV_ERR_INVALID;
   }

@@ -127,8 +127,20 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
 // ---------------------------------------------------------------------------
 // Partition: persistent grid, one stream-K worker per CTA, one KV head per warp.
 // ---------------------------------------------------------------------------
-// One lookahead entry: s, hg | nt << 12, j, flags, new_slot, len, phys[kMaxBoxes].
-constexpr int kEntryInts = 6 + kMaxBoxes;
+// One lookahead entry: s, hg | nt << 12, j, flags, new_slot, len, pair start
+// (flattened index of the pair's first tile), phys[kMaxBoxes].
+constexpr int kEntryInts = 7 + kMaxBoxes;
+
+// Per-warp values kept in shared memory rather than in registers of the
+// streaming loop.
+struct RangeInfo {
+  int32_t x0;  // flattened index of the range's first tile
+  // a written piece whose arrival waits: its request, head group, the pair's
+  // first tile (flattened) and tile count
+  int32_t pend_s, pend_hg, pend_pstart, pend_nt;
+  int32_t active_workers;  // the plan's worker count and tile total
+  long long total_tiles;
+};
 
 template <class Core, int W, int DEPTH>
 struct Smem {
@@ -138,8 +150,9 @@ struct Smem {
   static constexpr int kBatchInts = kBatch * kEntryInts;
   static constexpr int kBatchB = kBatchInts * 4;
   static constexpr int kBars = DEPTH * 8;
+  static constexpr int kInfo = int(sizeof(RangeInfo));
   static constexpr int kPerWarp =
-      round_up(kStages + kScratch + kMeta + kBatchB + kBars, Core::kAlign);
+      round_up(kStages + kScratch + kMeta + kBatchB + kBars + kInfo, Core::kAlign);
   static constexpr int kTotal = W * kPerWarp + Core::kAlign;  // + slack to align the base
 };
 
@@ -181,10 +194,18 @@ __global__ void __launch_bounds__(W * 32, CPS)
   StageMeta* meta = reinterpret_cast<StageMeta*>(wbase + SM::kStages + SM::kScratch);
   int32_t* bt = reinterpret_cast<int32_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta + SM::kBatchB);
+  RangeInfo* rinfo = reinterpret_cast<RangeInfo*>(wbase + SM::kStages + SM::kScratch + SM::kMeta + SM::kBatchB +
+                                                  SM::kBars);
 
   // The next kernel of the stream may be scheduled now; it starts on an SM
   // as this launch's CTAs leave it.
   if (threadIdx.x == 0) grid_launch_dependents();
+  if (blockIdx.x >= a.num_workers) {
+    // the extra CTA of an independent launch: it only keeps the launch from
+    // completing before the kernel ahead of it in the stream
+    grid_dependency_wait();
+    return;
+  }
   // Until grid_dependency_wait() below, this launch only reads what the
   // kernel just before it does not write (plan, tables, lengths, slots, K/V
   // pool), through L2, and writes no global memory but error flags.
@@ -193,13 +214,13 @@ __global__ void __launch_bounds__(W * 32, CPS)
   if (__ldcg(&hdr->planned) != 1 || __ldcg(&hdr->num_seqs) != check_S || __ldcg(&hdr->num_q_heads) != check_Hq ||
       __ldcg(&hdr->num_kv_heads) != check_Hkv || __ldcg(&hdr->head_dim) != check_D ||
       __ldcg(&hdr->kv_dtype) != check_dtype || __ldcg(&hdr->num_workers) != a.num_workers ||
-      __ldcg(&hdr->head_groups) != a.head_groups) {
+      __ldcg(&hdr->head_groups) != a.head_groups || __ldcg(&hdr->active_workers) < 1 ||
+      __ldcg(&hdr->active_workers) > a.num_workers) {
     grid_dependency_wait();
     if (threadIdx.x == 0) record_status(status, kStatusPlanMismatch);
     return;
   }
-  const long long TT = __ldcg(&hdr->total_tiles);
-  const int NW = a.num_workers;
+  const int NW = a.num_workers;  // CTAs of the grid (and partial-state slots)
   const int v = blockIdx.x;  // this CTA's worker id; warp = head within the group
   const int4 wp = __ldcg(reinterpret_cast<const int4*>(a.ws + a.off_wplan) + 2 * v);
   const int first_len = __ldcg(reinterpret_cast<const int4*>(a.ws + a.off_wplan) + 2 * v + 1).x;
@@ -241,6 +262,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
   // when the loads have long landed.  The cursor (request cs, offset coff in
   // its NHG * nt tiles, its length clen) is warp-uniform; seq_lens is only
   // read when the walk crosses into a new request.
+  if (lane == 0)
+    *rinfo = RangeInfo{wp.x, 0, 0, 0, 0, __ldcg(&hdr->active_workers), __ldcg(&hdr->total_tiles)};
+  __syncwarp();
   int cs = wp.z, coff = wp.w;
   int clen = first_len;
   int n_s = 0, n_hg = 0, n_j = 0, n_flags = 0, n_nt = 0, n_len = 0;
@@ -301,7 +325,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
     clen = __shfl_sync(0xffffffffu, clen, kBatch - 1);
   };
 
-  auto commit = [&]() {
+  auto commit = [&](int kb) {  // kb: the first processing step of the batch
     if (n_valid) {
       int32_t* e = bt + lane * kEntryInts;
       e[0] = n_s;
@@ -314,6 +338,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       else if (n_slot >= 0)
         e[4] = static_cast<int>(n_slot);
       if constexpr (MULTI) e[5] = n_len;
+      e[6] = rinfo->x0 + kb + lane - n_j;  // flattened index of the pair's first tile
 #pragma unroll
       for (int b = 0; b < kMaxBoxes; ++b) {
         int phys = -1;
@@ -326,7 +351,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
             phys = a.num_blocks;  // out of the tensor map: TMA fills zeros
           }
         }
-        e[6 + b] = phys;
+        e[7 + b] = phys;
       }
     }
     __syncwarp();
@@ -335,7 +360,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
   int last_s = -1, last_hg = -1;
   // q is written by earlier kernels: in the prologue (before the dependency
   // wait) a stage's q copy is held back, and the stage's arrival with it.
-  bool defer_q = true;
+  bool defer_q = !a.independent;
   uint32_t q_pending = 0;  // lane 0: stages whose q copy and arrival wait
   auto load_q = [&](int st, int s, int head) {
     char* stage = stages + st * Core::kStageBytes;
@@ -349,7 +374,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
   };
   auto issue = [&](int k) {
     if ((k % kBatch) == 0) {
-      commit();               // batch k, loaded during the previous batch
+      commit(k);              // batch k, loaded during the previous batch
       walk(k + kBatch);       // start loading batch k + kBatch
     }
     if (lane == 0) {
@@ -368,10 +393,11 @@ __global__ void __launch_bounds__(W * 32, CPS)
       meta[st].nt = e[1] >> 12;
       meta[st].new_slot = e[4];
       if constexpr (MULTI) meta[st].len = e[5];
+      meta[st].pstart = e[6];
       const uint32_t bar = smem_u32(&bars[st]);
       int nb = 0;
 #pragma unroll
-      for (int b = 0; b < kMaxBoxes; ++b) nb += (b < nbox && e[6 + b] >= 0) ? 1 : 0;
+      for (int b = 0; b < kMaxBoxes; ++b) nb += (b < nbox && e[7 + b] >= 0) ? 1 : 0;
       const uint32_t box_bytes = static_cast<uint32_t>(box_rows * Core::kChunkRowBytes);
       uint32_t bytes = 2u * nb * Core::kChunks * box_bytes;
       if (newpair) bytes += ncols * Core::ROWB;
@@ -386,7 +412,7 @@ __global__ void __launch_bounds__(W * 32, CPS)
       const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
 #pragma unroll
       for (int b = 0; b < kMaxBoxes; ++b) {
-        const int phys = e[6 + b];
+        const int phys = e[7 + b];
         if (b < nbox && phys >= 0) {
 #pragma unroll
           for (int c = 0; c < Core::kChunks; ++c) {
@@ -408,8 +434,8 @@ __global__ void __launch_bounds__(W * 32, CPS)
     for (int k = 0; k < prologue; ++k) issue(k);
   }
   // Everything below may read what earlier kernels wrote (q, k_new, v_new)
-  // and writes global memory.
-  grid_dependency_wait();
+  // and writes global memory.  An independent launch does not wait.
+  if (!a.independent) grid_dependency_wait();
   defer_q = false;
   if (lane == 0) {
     for (int st = 0; st < DEPTH; ++st) {
@@ -437,39 +463,115 @@ __global__ void __launch_bounds__(W * 32, CPS)
   typename Core::State state;
   bool have = false;
   int ps = 0, phg = 0, jfirst = 0, pnt = 0;
-  long long pstart = 0;
+  int pstart = 0;
   bool last_is_end = false;
 
-  auto flush = [&]() {
+  // Arrival of a finished piece of pair (request s_, head group hg_) on the
+  // pair's counter (lane 0; acquire-release at GPU scope: the release
+  // publishes the warp's partial writes, the acquire lets the last arrival
+  // see every other piece's).  Its result is read later, by last_piece().
+  auto count_in = [&](int s_, int hg_) {
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[static_cast<size_t>(s_) * Hkv + hg_ * W + warp], 1);
+    return prev;
+  };
+  // Whether an arrival that found `prev` earlier arrivals completed the pair
+  // whose first tile is pstart_ (pnt_ tiles).
+  auto last_piece = [&](int prev_lane0, int pstart_, int pnt_, int& v0, int& v1, long long& TT, int& NWa) {
+    const int prev = __shfl_sync(0xffffffffu, prev_lane0, 0);
+    // the plan's totals, kept in shared memory rather than in registers of the loop
+    TT = rinfo->total_tiles;
+    NWa = rinfo->active_workers;  // workers the tiles are split over
+    v0 = owner_of(pstart_, TT, NWa);
+    v1 = owner_of(pstart_ + pnt_ - 1, TT, NWa);
+    int expected = v1 - v0 + 1;  // with TT >= NWa every active CTA owns at least one tile
+    if (TT < NWa) {
+      expected = 0;
+      for (int u = v0; u <= v1; ++u) expected += range_begin(u, TT, NWa) < range_begin(u + 1, TT, NWa) ? 1 : 0;
+    }
+    return prev == expected - 1;
+  };
+  // Merge the partial states of a completed pair and clear its counter.
+  auto merge = [&](int s_, int hg_, int v0, int v1, long long TT, int NWa) {
+    const int head = hg_ * W + warp;
+    const OutMap om{(static_cast<size_t>(s_) * T * Hq + static_cast<size_t>(head) * Gq) * D,
+                    static_cast<size_t>(Hq) * D, Gq, D, ncols};
+    const long long pp = static_cast<long long>(s_) * NHG + hg_;  // pair index
+    __syncwarp();  // lane 0's acquire orders the whole warp's loads (barrier semantics)
+    merge_pair<D, G, W, MULTI>(partials, pp, warp, v0, v1, TT, NWa, a.out, a.out_dtype, om, lane);
+    if (lane == 0) atomicExch(&counters[static_cast<size_t>(s_) * Hkv + head], 0);
+  };
+
+  // A range holds at most two pieces of split pairs: the first pair (begun by
+  // an earlier CTA) and the last (continued by a later one); every pair in
+  // between is whole and written directly.  The first piece's partial state is
+  // written when the warp moves on to the next pair, but its arrival is
+  // issued one tile later (by then the partial writes have reached L2, so
+  // the release costs no wait) and its result read one tile after that (the
+  // atomic's round trip overlaps the stream).  In the rare case that this
+  // arrival completes the pair, the merge waits for the end of the range.
+  int pend = 0;       // 1: piece written, arrival not issued; 2: arrival issued, result not read
+  int pend_prev = 0;  // lane 0: result of the delayed arrival
+  bool pend_merge = false;  // the delayed arrival completed its pair: merge at the end
+  auto settle = [&](bool to_end) {  // advance the delayed arrival (to completion if to_end)
+    if (pend == 1) {
+      pend_prev = count_in(rinfo->pend_s, rinfo->pend_hg);
+      pend = 2;
+      if (!to_end) return;
+    }
+    if (pend == 2) {
+      int v0, v1, NWa;
+      long long TT;
+      pend_merge = last_piece(pend_prev, rinfo->pend_pstart, rinfo->pend_nt, v0, v1, TT, NWa);
+      pend = 0;
+    }
+  };
+  auto merge_pending = [&]() {
+    if (!pend_merge) return;
+    int v0, v1, NWa;
+    long long TT;
+    last_piece(0, rinfo->pend_pstart, rinfo->pend_nt, v0, v1, TT, NWa);
+    merge(rinfo->pend_s, rinfo->pend_hg, v0, v1, TT, NWa);
+    pend_merge = false;
+  };
+  auto flush = [&](bool final) {
     const int head = phg * W + warp;
     const OutMap om{(static_cast<size_t>(ps) * T * Hq + static_cast<size_t>(head) * Gq) * D,
                     static_cast<size_t>(Hq) * D, Gq, D, ncols};
     float* const lse = MULTI ? a.lse : nullptr;
-    if (jfirst == 0 && last_is_end) {  // the whole pair is in this CTA's range
+    const bool whole = jfirst == 0 && last_is_end;  // the whole pair is in this CTA's range
+    if (whole) {
       Core::finish(state, true, a.out, a.out_dtype, om, nullptr, lane, lse);
+    } else {
+      const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
+      float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
+      Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
+    }
+    if (!final && !whole) {
+      // (a second such piece cannot occur; should it, the first one settles now)
+      settle(true);
+      merge_pending();
+      __syncwarp();
+      if (lane == 0) {
+        rinfo->pend_s = ps;
+        rinfo->pend_hg = phg;
+        rinfo->pend_pstart = pstart;
+        rinfo->pend_nt = pnt;
+      }
+      __syncwarp();
+      pend = 1;
       return;
     }
-    const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
-    float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
-    Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
-    // Count this CTA in for (request, KV head); the last CTA of the pair merges.
-    const size_t ctr = static_cast<size_t>(ps) * Hkv + head;
-    // Release the warp's partial writes and count in (acquire-release at GPU
-    // scope: the last arrival sees every other CTA's partial state).
-    __syncwarp();
-    int prev = 0;
-    if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[ctr], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + pnt - 1, TT, NW);
-    int expected = v1 - v0 + 1;  // with TT >= NW every CTA owns at least one tile
-    if (TT < NW) {
-      expected = 0;
-      for (int u = v0; u <= v1; ++u) expected += range_begin(u, TT, NW) < range_begin(u + 1, TT, NW) ? 1 : 0;
-    }
-    if (prev == expected - 1) {
-      __syncwarp();  // lane 0's acquire orders the whole warp's loads (barrier semantics)
-      merge_pair<D, G, W, MULTI>(partials, pp, warp, v0, v1, TT, NW, a.out, a.out_dtype, om, lane);
-      if (lane == 0) atomicExch(&counters[ctr], 0);
+    if (final) {
+      settle(true);
+      if (!whole) {
+        const int prev = count_in(ps, phg);
+        int v0, v1, NWa;
+        long long TT;
+        if (last_piece(prev, pstart, pnt, v0, v1, TT, NWa)) merge(ps, phg, v0, v1, TT, NWa);
+      }
+      merge_pending();
     }
   };
 
@@ -477,18 +579,25 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const int st = k % DEPTH;
     if (!mbar_wait_bounded(smem_u32(&bars[st]), (k / DEPTH) & 1)) {
       if (lane == 0) record_status(status, kStatusTimeout);
+      // Stop computing and issue no new copies, but give the copies already
+      // issued into this warp's ring (tiles k .. k + DEPTH - 1) a last short
+      // wait each before the CTA exits, so none lands in shared memory that a
+      // newly scheduled CTA already uses.  A copy that has not landed after
+      // that second limit is taken as lost; the status word reports the launch.
+      for (int kk = k; kk < ntiles && kk < k + DEPTH; ++kk)
+        mbar_wait_bounded(smem_u32(&bars[kk % DEPTH]), (kk / DEPTH) & 1, kDrainLimitNs);
       return;
     }
     const StageMeta m = meta[st];
     const char* stage = stages + st * Core::kStageBytes;
     if (m.flags & 1) {
-      if (have) flush();
+      if (have) flush(false);
       have = true;
       ps = m.s;
       phg = m.hg;
       jfirst = m.j;
       pnt = m.nt;
-      pstart = static_cast<long long>(wp.x) + k - m.j;
+      pstart = m.pstart;
       Core::begin_pair(state, stage + Core::kQOff, a.scale_log2, lane);
     }
     const int nvalid = m.flags >> 8;
@@ -519,8 +628,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
     }
     __syncwarp();
     if (k + DEPTH < ntiles) issue(k + DEPTH);
+    if (pend != 0) settle(false);
   }
-  if (have) flush();
+  if (have) flush(true);
 }
 
 
@@ -560,15 +670,21 @@ int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
+    // Every variant asks for the largest shared-memory carve-out, so CTAs of
+    // two different variants (launches that overlap) can share an SM without
+    // it first draining to reconfigure its L1 / shared split.
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return host::cuda_fail(e);
     configured_dev = dev;
   }
+  const int grid = geo.NW + (args.independent ? 1 : 0);
   if (!geo.overlap) {
-    kern<<<geo.NW, W * 32, SM::kTotal, stream>>>(maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
+    kern<<<grid, W * 32, SM::kTotal, stream>>>(maps, args, geo.S, geo.Hq, geo.Hkv, geo.D, geo.dtype);
     return host::check_launch();
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(geo.NW);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(W * 32);
   cfg.dynamicSmemBytes = SM::kTotal;
   cfg.stream = stream;

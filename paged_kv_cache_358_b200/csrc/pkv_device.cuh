@@ -22,6 +22,8 @@ enum : uint32_t {
 // enough never to trigger on a healthy launch (a tile lands in microseconds),
 // short enough that a broken pipeline ends the launch instead of hanging it.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// After a timeout, each copy still in flight gets this much longer.
+constexpr uint64_t kDrainLimitNs = 50000000ull;    // 50 ms
 
 PKV_DEVINL uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

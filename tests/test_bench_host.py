@@ -25,12 +25,24 @@ def test_step_bytes_count_each_history_slot_once_per_kv_head():
     assert 32 * 32 * 4096 * 8 * 128 * 2 * 2 == 16 * 2 ** 30
 
 
-def test_copy_on_write_bytes_are_added_per_layer():
+def test_copy_on_write_bytes_count_the_valid_rows_per_layer():
+    """A copy-on-write moves n_valid = n mod B rows of K and V (read and written)
+    in every layer, not the whole block: three copies of 8, 1 and 15 rows."""
     d = _dummy()
     lens = np.full(32, 100, dtype=np.int64)
     base = bench.DecodeStep.bytes_of_step(d, lens, 0)
-    with_cow = bench.DecodeStep.bytes_of_step(d, lens, 3)
-    assert with_cow - base == 32 * 3 * 16 * 8 * 128 * 2 * 2 * 2
+    with_cow = bench.DecodeStep.bytes_of_step(d, lens, 8 + 1 + 15)
+    row = 8 * 128 * 2                                   # one token of one layer's K (or V) pool
+    assert with_cow - base == 32 * (8 + 1 + 15) * row * 2 * 2
+    assert with_cow - base < 32 * 3 * 16 * row * 2 * 2  # less than three whole blocks
+
+
+def test_step_stats_are_order_statistics():
+    x = [3.0, 1.0, 2.0, 10.0, 4.0]
+    st = bench.step_stats(x)
+    assert st["median"] == 3.0 and st["n"] == 5
+    assert st["p10"] == np.percentile(x, 10) and st["p90"] == np.percentile(x, 90)
+    assert st["mean"] == 4.0
 
 
 def test_traffic_file_is_read_by_key():

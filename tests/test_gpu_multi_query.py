@@ -47,7 +47,7 @@ def _ref(hb, q):
 
 @pytest.mark.parametrize("T,Hq,Hkv,D,B,dtype", [
     (2, 32, 8, 128, 16, "bf16"),   # 8 columns per KV head: tensor-core tiles
-    (4, 32, 8, 128, 16, "bf16"),   # 16 columns: CUDA-core tiles
+    (4, 32, 8, 128, 16, "bf16"),   # 16 columns: columns-in-M tensor-core tiles (CUDA-core when forced)
     (3, 8, 4, 64, 8, "bf16"),      # 6 columns padded to 8
     (5, 4, 4, 256, 32, "bf16"),    # 5 columns padded to 8, 512-byte rows
     (3, 16, 4, 64, 16, "f32"),     # 12 columns padded to 16, fp32 pools

@@ -136,6 +136,21 @@ def test_shared_prefix_flags_a_false_claim():
                                         torch.from_numpy(lens).cuda(), torch.from_numpy(gs).cuda(),
                                         torch.from_numpy(pb).cuda(), 2, 1.0 / np.sqrt(D), workspace=ws)
     assert pkv.decode_status(ws) == pkv.Status.BAD_TABLE
+    # a fault of an earlier call is not reported again: a valid call on the
+    # same workspace (its shared-part status word included) reports OK, and
+    # so does a valid call on a workspace full of stale bytes
+    pb_ok = np.array([40 // B, 0], np.int32)
+    for fill in (None, 0xFF):
+        if fill is not None:
+            ws.fill_(fill)
+        out = pkv.paged_decode_attn_shared_prefix(torch_from_host(q), kp, vp, torch.from_numpy(tables).cuda(),
+                                                  torch.from_numpy(lens).cuda(), torch.from_numpy(gs).cuda(),
+                                                  torch.from_numpy(pb_ok).cuda(), 2, 1.0 / np.sqrt(D),
+                                                  out_dtype=torch.float32, workspace=ws)
+        assert pkv.decode_status(ws) == pkv.Status.OK
+        got = as_f64(out)
+        for s in range(4):
+            assert np.max(np.abs(got[s] - oatt.dense_decode(q[s], hk[s], hv[s], 1.0 / np.sqrt(D)))) <= 1e-2
 
 
 def test_shared_prefix_rejects_unsupported_groups():

@@ -5,9 +5,10 @@ memory themselves (a plugin whose host runtime owns every device allocation,
 a serving loop that must never call cudaMalloc).  It keeps its scratch in an
 array built into the library, shared by every call on a device.  This test
 calls it through the C ABI twice in a row, on two different batches, and
-checks each result against pkv_paged_decode_attn with a caller workspace, so
-a second call that picked up state left by the first would fail.  It also
-checks that a batch too large for the built-in scratch is refused.
+checks each result against pkv_paged_decode_attn with a caller workspace and
+against the float64 oracle, so a second call that picked up state left by the
+first would fail.  It also checks that a batch whose stated workspace size is
+beyond the built-in scratch is refused, for both storage types.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it passes alone in a fresh process as well.
@@ -18,7 +19,7 @@ import numpy as np
 import pytest
 
 import workloads as W
-from tests.paged_batch import as_f64, device_batch, host_batch
+from tests.paged_batch import as_f64, device_batch, host_batch, oracle_out
 
 pytestmark = pytest.mark.gpu
 
@@ -54,21 +55,43 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         g, r = as_f64(got), as_f64(ref)
         assert np.all(np.isfinite(g))
         assert np.max(np.abs(g - r)) <= tol
+        assert np.max(np.abs(g - oracle_out(hb))) <= tol
 
 
-def test_noalloc_refuses_batches_beyond_its_scratch():
+@pytest.mark.parametrize("kv_dtype", ["bf16", "f32"])
+def test_noalloc_refuses_batches_beyond_its_scratch(kv_dtype):
     import torch
 
     import paged_kv_cache_358_b200 as pkv
 
-    S, Hq, Hkv, D = 8192, 32, 8, 128
-    assert pkv.decode_workspace_bytes(S, Hq, Hkv, D) > (16 << 20)
-    q = torch.zeros((1, Hq, D), dtype=torch.bfloat16, device="cuda")
-    pool = torch.zeros((4, 16, Hkv, D), dtype=torch.bfloat16, device="cuda")
-    t = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
-    out = torch.zeros((1, Hq, D), dtype=torch.float32, device="cuda")
+    Hq, Hkv, D = 32, 8, 128
+    # the smallest batch whose stated workspace size exceeds 16 MiB is refused,
+    # the largest one within it runs
+    lo, hi = 1, 1 << 16
+    while lo < hi:
+        mid = (lo + hi) // 2
+        if pkv.decode_workspace_bytes(mid, Hq, Hkv, D) > (16 << 20):
+            hi = mid
+        else:
+            lo = mid + 1
+    S_over = lo
+    assert pkv.decode_workspace_bytes(S_over - 1, Hq, Hkv, D) <= (16 << 20)
+    dt = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
+    code = pkv.BF16 if kv_dtype == "bf16" else pkv.F32
+    q = torch.zeros((S_over, Hq, D), dtype=dt, device="cuda")
+    pool = torch.zeros((4, 16, Hkv, D), dtype=dt, device="cuda")
+    t = torch.zeros((S_over, 1), dtype=torch.int32, device="cuda")
+    lens = torch.zeros((S_over,), dtype=torch.int32, device="cuda")
+    out = torch.full((S_over, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
     rc = pkv.lib().pkv_paged_decode_attn_noalloc(
-        q.data_ptr(), pool.data_ptr(), pool.data_ptr(), t.data_ptr(), 1, t.data_ptr(), S, Hq, Hkv, D, 16, 4,
-        ctypes.c_float(0.1), pkv.BF16, out.data_ptr(), pkv.F32, None)
+        q.data_ptr(), pool.data_ptr(), pool.data_ptr(), t.data_ptr(), 1, lens.data_ptr(), S_over, Hq, Hkv, D, 16,
+        4, ctypes.c_float(0.1), code, out.data_ptr(), pkv.F32, None)
     assert rc == pkv.Status.INVALID
     assert "16 MiB" in pkv.lib().pkv_last_cuda_error().decode()
+    # one request fewer fits: every length is 0, so every output is 0
+    rc = pkv.lib().pkv_paged_decode_attn_noalloc(
+        q.data_ptr(), pool.data_ptr(), pool.data_ptr(), t.data_ptr(), 1, lens.data_ptr(), S_over - 1, Hq, Hkv, D,
+        16, 4, ctypes.c_float(0.1), code, out.data_ptr(), pkv.F32, None)
+    assert rc == pkv.Status.OK
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out[:S_over - 1]).item() == 0
