@@ -32,45 +32,11 @@ struct PlanArgs {
   int S, Hq, Hkv, NHG, D, kv_dtype, NW;
   char* ws;
   size_t off_prefix, off_wplan, off_counters;
-  int cost;  // relative cost of one of this plan's tiles (two plans sharing the SMs)
 };
 
-// Workers of the first of two launches that run side by side and share the
-// NW worker slots: proportional to the launches' costs (tiles x cost per
-// tile), at least one each when both have work.
-__device__ __forceinline__ int split_workers(long long tiles0, int cost0, long long tiles1, int cost1, int NW) {
-  const long long w0 = tiles0 * cost0, w1 = tiles1 * cost1;
-  if (w1 == 0) return NW;
-  if (w0 == 0) return 0;
-  long long n0 = (w0 * NW + (w0 + w1) / 2) / (w0 + w1);
-  if (n0 < 1) n0 = 1;
-  if (n0 > NW - 1) n0 = NW - 1;
-  return static_cast<int>(n0);
-}
-
-// Tiles of a request-length array (block reduction over one CTA), times NHG.
-__device__ long long block_total_tiles(const int32_t* __restrict__ seq_lens, int S, int NHG) {
-  __shared__ long long part[kPlanThreads / 32];
-  long long x = 0;
-  for (int s = threadIdx.x; s < S; s += kPlanThreads) x += ntiles_of(seq_lens[s]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = x;
-  __syncthreads();
-  long long t = 0;
-  for (int w = 0; w < kPlanThreads / 32; ++w) t += part[w];
-  __syncthreads();
-  return t * NHG;
-}
-
-// NWa: the tiles are split over workers 0 .. NWa-1 (NWa <= NW, or a negative
-// value: compute it from `other`, a second plan whose launch runs side by side
-// with this one; `first` says which of the two this is).
 __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int S, int Hq, int Hkv,
                                           int NHG, int D, int kv_dtype, int NW, char* ws, size_t off_prefix,
-                                          size_t off_wplan, size_t off_counters, int NWa = -1,
-                                          const PlanArgs* self = nullptr, const PlanArgs* other = nullptr,
-                                          bool first = true) {
+                                          size_t off_wplan, size_t off_counters) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + off_prefix);
   int4* wplan = reinterpret_cast<int4*>(ws + off_wplan);
@@ -122,25 +88,17 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   __syncthreads();
   const long long T = total_seq_tiles * NHG;
   const int32_t* P = in_smem ? sp : prefix;
-  if (other != nullptr) {
-    const long long To = block_total_tiles(other->seq_lens, other->S, other->NHG);
-    const int n_first = first ? split_workers(T, self->cost, To, other->cost, NW)
-                              : split_workers(To, other->cost, T, self->cost, NW);
-    NWa = first ? n_first : NW - n_first;
-  }
-  if (NWa < 1 || NWa > NW) NWa = NWa < 1 ? 1 : NW;
 
-  // Worker v < NWa owns tiles [floor(v T / NWa), floor((v+1) T / NWa)); its
-  // first request is the last s with NHG * P[s] <= start (skipping empty
-  // requests).  Workers NWa .. NW-1 own none.
+  // Worker v owns tiles [floor(v T / NW), floor((v+1) T / NW)); its first
+  // request is the last s with NHG * P[s] <= start (skipping empty requests).
   for (int v = tid; v < NW; v += kPlanThreads) {
-    if (T == 0 || v >= NWa) {
+    if (T == 0) {
       wplan[2 * v] = make_int4(0, 0, 0, 0);
       wplan[2 * v + 1] = make_int4(0, 0, 0, 0);
       continue;
     }
-    const long long a = range_begin(v, T, NWa);
-    const long long b = range_begin(v + 1, T, NWa);
+    const long long a = range_begin(v, T, NW);
+    const long long b = range_begin(v + 1, T, NW);
     int lo = 0, hi = S - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -157,7 +115,6 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
     hdr->head_dim = D;
     hdr->kv_dtype = kv_dtype;
     hdr->num_workers = NW;
-    hdr->active_workers = NWa;
     hdr->head_groups = NHG;
     hdr->total_tiles = T;
     hdr->planned = 1;
@@ -169,16 +126,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int kv_dtype, int NW, char* ws,
                                                             size_t off_prefix, size_t off_wplan,
                                                             size_t off_counters) {
-  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters, NW);
+  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters);
 }
 
-// The plans of two launches that run side by side, one per CTA: the two
-// launches split the worker slots in proportion to their costs.
+// Two independent plans in one launch, one per CTA.
 __global__ void __launch_bounds__(kPlanThreads) plan2_kernel(const PlanArgs p0, const PlanArgs p1) {
-  const bool first = blockIdx.x == 0;
-  const PlanArgs& p = first ? p0 : p1;
+  const PlanArgs& p = blockIdx.x == 0 ? p0 : p1;
   plan_body(p.seq_lens, p.S, p.Hq, p.Hkv, p.NHG, p.D, p.kv_dtype, p.NW, p.ws, p.off_prefix, p.off_wplan,
-            p.off_counters, -1, &p, first ? &p1 : &p0, first);
+            p.off_counters);
 }
 
 }  // namespace pkv
@@ -362,8 +317,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
-             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr,
-             int32_t independent = 0) {
+             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -404,7 +358,6 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.num_q_tokens = num_q_tokens;
   args.causal = causal;
   args.lse = lse;
-  args.independent = independent;
   geo.overlap = overlap;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
@@ -699,16 +652,13 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
   // both plans in one launch
-  // The two passes run side by side and share the worker slots in
-  // proportion to their tiles, a shared-part tile (16 columns) costing about
-  // 1.35 times an own-part tile (the grouped heads of one query).
-  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws, int cost) {
+  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws) {
     return PlanArgs{lens, g.S, g.Hq, g.Hkv, g.NHG, g.D, g.dtype, g.NW, pws,
-                    g.lay.prefix, g.lay.wplan, g.lay.counters, cost};
+                    g.lay.prefix, g.lay.wplan, g.lay.counters};
   };
   plan2_kernel<<<2, kPlanThreads, 0, st>>>(
-      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws, 20),
-      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws, 27));
+      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws),
+      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws));
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
   // own-part pass: each request over its own blocks
@@ -718,19 +668,15 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                 stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
   if (rc != PKV_OK) return rc;
   // shared-part pass: groups x members, every member sees the whole shared
-  // part.  It runs side by side with the own-part pass (a programmatic
-  // dependent launch that never waits for it, on the worker slots the own-part
-  // plan leaves idle): everything it reads -- its plan, the grouped queries,
-  // the group tables and lengths, the pools -- was written by the gather and
-  // plan kernels, which finished before the own-part pass began, and it
-  // writes only its own workspace, o_p and lse_p, which the own-part pass
-  // does not touch.  Its one extra CTA waits for the own-part pass, so the
-  // combine kernel after it sees both results.
+  // part.  It may start during the own-part pass's tail (launch overlap):
+  // what it reads first -- its plan, the group tables and lengths, the pools
+  // -- was written by the gather and plan kernels, which finished before
+  // the own-part pass began; that pass writes only its own workspace and o_s.
   rc = run_impl(w + c.q_grp, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.grp_table),
                 max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
                 num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
                 w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, true, 0,
-                reinterpret_cast<float*>(w + c.lse_p), 1);
+                reinterpret_cast<float*>(w + c.lse_p));
   if (rc != PKV_OK) return rc;
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
   const int threads = 256;

@@ -44,7 +44,7 @@ struct WsHeader {
   int32_t num_workers;     // CTAs of the partition grid
   int32_t head_groups;     // KV-head groups per request
   int32_t planned;
-  int32_t active_workers;  // workers the tiles are split over (<= num_workers; the rest idle)
+  int32_t pad;
   long long total_tiles;   // flattened (request, head group, tile) units
 };
 
@@ -54,9 +54,9 @@ constexpr int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
 
 // Workspace layout (byte offsets, each 256-aligned):
 //   header | prefix int32[S+1] (tiles per request, cumulative) |
-//   worker plan int4[2*NW] {tile_begin, tile_end, s, offset in s}, {len(s), 0, 0, 0}
-//     (the tiles are split over the first active_workers <= NW workers) |
-//   arrival counters int32[S*H_kv] (CTAs done with a split (request, KV head)) |
+//   worker plan int4[2*NW] {tile_begin, tile_end, s, offset in s}, {len(s), 0, 0, 0} |
+//   arrival counters int32[S*H_kv] (pieces of a split (request, KV head) counted in: low 16
+//     bits those that ended their CTA's range, high 16 bits the one flushed mid-range) |
 //   partial states float[(NW + S*NHG) * HG][part_stride(G, D)]
 struct WsLayout {
   size_t prefix = 0, wplan = 0, counters = 0, partials = 0, total = 0;
@@ -88,10 +88,6 @@ struct DecodeArgs {
   int32_t num_workers;
   int32_t num_q_tokens;  // T query tokens per request (1 for plain decode)
   int32_t causal;        // T > 1: 1 = token i sees positions < len - (T-1-i); 0 = all see all
-  // 1: the launch reads and writes nothing the kernel before it in the stream
-  // writes or reads, so its workers never wait for that kernel; one extra CTA
-  // (index num_workers) waits for it, so this launch still completes after it.
-  int32_t independent;
   float scale_log2;     // scale * log2(e)
   // Optional log-sum-exp output (null: none): lse[s][i][h] = log2 of the
   // softmax denominator in the log2 domain of the scores (-inf when nothing
@@ -180,7 +176,7 @@ struct alignas(16) StageMeta {
   int32_t nt;      // tiles of the pair
   int32_t new_slot;  // folded append: pool slot of the pair's new token (< 0: none)
   int32_t len;       // length of the request
-  int32_t pstart;    // flattened index of the pair's first tile
+  int32_t pad;
 };
 
 }  // namespace pkv

@@ -17,9 +17,9 @@
 // score accumulator (token-major) is turned into the P^T operand of the value
 // MMA with movmatrix.trans, after the online-softmax update of [P3] eq. (4)
 // in fp32 on the accumulator registers.  P is rounded to bf16 for the value
-// MMA (relative error <= 2^-9 per weight) and the running sum l adds the same
-// rounded weights, so the output is an exactly normalised average of V;
-// everything else stays fp32.
+// MMA (relative error <= 2^-9 per weight) while the running sum l adds the
+// fp32 weights, so the output's scale is off by at most 2^-9; everything
+// else stays fp32.
 // Slots at or past the length: their scores are replaced by -inf, and in the
 // last tile their V^T operand columns are zeroed before the MMA, so stale NaN
 // rows cannot reach the accumulator through 0 * NaN.
@@ -127,8 +127,8 @@ struct MmaCore {
     const int gid = lane >> 2, tig = lane & 3;
     const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
 
-    // scores S^T = K Q^T, the k-steps split over two accumulators (even and
-    // odd steps) so the dependent MMA chain is half as long
+    // scores S^T = K Q^T, the k-steps alternating between two accumulators so
+    // the dependent MMA chain is half as long
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     {
       float c2[4] = {0.f, 0.f, 0.f, 0.f};
@@ -166,16 +166,13 @@ struct MmaCore {
       r0 = mn0 == -INFINITY ? 0.f : mn0;
       r1 = mn1 == -INFINITY ? 0.f : mn1;
     }
-    const float al0 = exp2f(st.m[0] - r0), al1 = exp2f(st.m[1] - r1);
+    const float al0 = fast_exp2(st.m[0] - r0), al1 = fast_exp2(st.m[1] - r1);
     st.m[0] = mn0;
     st.m[1] = mn1;
-    const float p0 = exp2f(s[0] - r0), p1 = exp2f(s[1] - r1);
-    const float p2 = exp2f(s[2] - r0), p3 = exp2f(s[3] - r1);
-    // the weights as the value MMA sees them (bf16); the running sum adds the
-    // same rounded weights, so the output is their exact normalised average
-    const uint32_t pk0 = pack_bf16x2(p0, p1), pk1 = pack_bf16x2(p2, p3);
-    st.l[0] = st.l[0] * al0 + (bf16lo(pk0) + bf16lo(pk1));
-    st.l[1] = st.l[1] * al1 + (bf16hi(pk0) + bf16hi(pk1));
+    const float p0 = fast_exp2(s[0] - r0), p1 = fast_exp2(s[1] - r1);
+    const float p2 = fast_exp2(s[2] - r0), p3 = fast_exp2(s[3] - r1);
+    st.l[0] = st.l[0] * al0 + (p0 + p2);
+    st.l[1] = st.l[1] * al1 + (p1 + p3);
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
       for (int mt = 0; mt < KSTEPS; ++mt) {
@@ -186,8 +183,8 @@ struct MmaCore {
       }
     }
     // P^T operand: transpose the token-major fragments
-    const uint32_t b0 = movmatrix_trans(pk0);
-    const uint32_t b1 = movmatrix_trans(pk1);
+    const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
 
     // values O^T += V^T P^T
     const int vt = ((lane >> 4) << 3) + (lane & 7);
@@ -340,12 +337,9 @@ struct MmaCoreM16 {
     const int gid = lane >> 2, tig = lane & 3;
     const uint32_t kbase = smem_u32(ksm), vbase = smem_u32(vsm);
 
-    // scores: s0 for tokens 0..7, s1 for tokens 8..15 (C rows = columns); the
-    // k-steps alternate between two accumulators each, so the dependent MMA
-    // chains are half as long
+    // scores: s0 for tokens 0..7, s1 for tokens 8..15 (C rows = columns)
     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
     {
-      float s0b[4] = {0.f, 0.f, 0.f, 0.f}, s1b[4] = {0.f, 0.f, 0.f, 0.f};
       // matrices: (tok 0-7, unit 2kk), (tok 0-7, 2kk+1), (tok 8-15, 2kk), (tok 8-15, 2kk+1)
       const int t = (lane & 7) + ((lane >> 4) << 3);
       const int hu = (lane >> 3) & 1;
@@ -353,13 +347,8 @@ struct MmaCoreM16 {
       for (int kk = 0; kk < KSTEPS; ++kk) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kbase + swz(t, 2 * kk + hu), b0, b1, b2, b3);
-        mma_bf16_16816((kk & 1) ? s0b : s0, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b0, b1);
-        mma_bf16_16816((kk & 1) ? s1b : s1, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b2, b3);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        s0[i] += s0b[i];
-        s1[i] += s1b[i];
+        mma_bf16_16816(s0, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b0, b1);
+        mma_bf16_16816(s1, st.qa[kk][0], st.qa[kk][1], st.qa[kk][2], st.qa[kk][3], b2, b3);
       }
     }
     // row gid: s0[0], s0[1], s1[0], s1[1] (tokens 2tig, 2tig+1, 8+2tig, 9+2tig); row gid+8: [2], [3]
@@ -387,23 +376,17 @@ struct MmaCoreM16 {
       r0 = mn0 == -INFINITY ? 0.f : mn0;
       r1 = mn1 == -INFINITY ? 0.f : mn1;
     }
-    const float al0 = exp2f(st.m[0] - r0), al1 = exp2f(st.m[1] - r1);
+    const float al0 = fast_exp2(st.m[0] - r0), al1 = fast_exp2(st.m[1] - r1);
     st.m[0] = mn0;
     st.m[1] = mn1;
     float p[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      p[i] = exp2f(x[i] - r0);
-      p[4 + i] = exp2f(x[4 + i] - r1);
+      p[i] = fast_exp2(x[i] - r0);
+      p[4 + i] = fast_exp2(x[4 + i] - r1);
     }
-    // P as the A operand (bf16): rows gid / gid+8, tokens 2tig(+1) and 8+2tig(+1);
-    // the running sums add these rounded weights, as the value MMA sees them
-    const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
-    const uint32_t pa1 = pack_bf16x2(p[4], p[5]);
-    const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
-    const uint32_t pa3 = pack_bf16x2(p[6], p[7]);
-    st.l[0] = st.l[0] * al0 + ((bf16lo(pa0) + bf16hi(pa0)) + (bf16lo(pa2) + bf16hi(pa2)));
-    st.l[1] = st.l[1] * al1 + ((bf16lo(pa1) + bf16hi(pa1)) + (bf16lo(pa3) + bf16hi(pa3)));
+    st.l[0] = st.l[0] * al0 + ((p[0] + p[1]) + (p[2] + p[3]));
+    st.l[1] = st.l[1] * al1 + ((p[4] + p[5]) + (p[6] + p[7]));
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -413,6 +396,11 @@ struct MmaCoreM16 {
         st.o[nt][3] *= al1;
       }
     }
+    // P as the A operand: rows gid / gid+8, tokens 2tig(+1) and 8+2tig(+1)
+    const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
+    const uint32_t pa1 = pack_bf16x2(p[4], p[5]);
+    const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
+    const uint32_t pa3 = pack_bf16x2(p[6], p[7]);
 
     // values: V as the B operand via ldmatrix.trans; matrices (tok 0-7, unit
     // 2mt), (tok 8-15, 2mt), (tok 0-7, 2mt+1), (tok 8-15, 2mt+1)

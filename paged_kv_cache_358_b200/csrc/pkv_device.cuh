@@ -25,6 +25,15 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // After a timeout, each copy still in flight gets this much longer.
 constexpr uint64_t kDrainLimitNs = 50000000ull;    // 50 ms
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error
+// below 2^-22; -inf gives +0).  The softmax weights it feeds are rounded to
+// bf16 (2^-9) before they multiply V.
+PKV_DEVINL float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 PKV_DEVINL uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -117,6 +126,18 @@ PKV_DEVINL void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_
           dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// Reduction (no value returned) with release semantics at GPU scope: the
+// thread's earlier writes are visible before the addition.
+PKV_DEVINL void red_release_gpu_add(unsigned* addr, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+// Load with acquire semantics at GPU scope.
+PKV_DEVINL unsigned ld_acquire_gpu(const unsigned* addr) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
 }
 
 // Atomic add with acquire-release semantics at GPU scope.

@@ -447,3 +447,29 @@ def test_bounded_device_wait_reports_timeout():
     got = as_f64(_run(db, hb, torch.float32))
     from tests.paged_batch import oracle_out
     assert np.max(np.abs(got - oracle_out(hb))) <= TOL_F32
+
+
+@pytest.mark.parametrize("G,D", [(4, 128), (16, 128), (8, 64)])
+def test_bf16_weight_rounding_bias_is_bounded(G, D):
+    """On the tensor-core tiles the softmax weights enter the P.V product
+    rounded to bf16 (relative error <= 2^-9 each) while the running sum adds
+    the unrounded fp32 weights, so the output's scale may be off by up to 2^-9
+    (a documented bound, well inside the 1e-2 budget).  With every V row equal
+    to 1 the exact output is exactly 1; the measured deviation must stay
+    within 2^-9 (plus fp32 accumulation), for the 4-, 8- and 16-column cores."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    Hkv = 4
+    wl = W.DecodeWorkload("ones", 1, G * Hkv, Hkv, D, 16, "bf16", (1, 15, 16, 300, 4097), pool_blocks=400, seed=31)
+    hb = host_batch(wl, q_scale=3.0)
+    for v in hb.v_hist:
+        v[...] = 0x3F80                       # bf16 1.0
+    db = device_batch(hb)
+    out = pkv.paged_decode_attn(db.q, db.k_pool, db.v_pool, db.tables, db.seq_lens, wl.scale,
+                                out_dtype=torch.float32)
+    got = as_f64(out)
+    dev = np.abs(got - 1.0)
+    assert np.all(np.isfinite(got))
+    assert dev.max() <= 2.0 ** -9 + 1e-6, dev.max()
