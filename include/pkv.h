@@ -247,10 +247,8 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  *                 meaningful)
  * Other arguments as pkv_paged_decode_attn.  Five launches: a gather, both
  * plans, the own-part pass, the shared-part pass (the members' queries are
- * the columns of one launch), and the combine.  The two passes run side by
- * side: the plans split the SMs' worker slots between them in proportion to
- * their tiles, and the shared-part pass, which reads nothing the own-part
- * pass writes, starts without waiting for it. */
+ * the columns of one launch; it starts during the own-part pass's tail), and
+ * the combine. */
 size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_blocks_per_seq);
