@@ -27,14 +27,9 @@ namespace pkv {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanSmemSeqs = 8192;  // prefix kept in shared memory up to this many requests
 
-struct PlanArgs {
-  const int32_t* seq_lens;
-  int S, Hq, Hkv, NHG, D, kv_dtype, NW;
-  char* ws;
-  size_t off_prefix, off_wplan, off_counters;
-};
-
-__device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int S, int Hq, int Hkv,
+// len_of(s): the length of request s (read from an array, or computed).
+template <class LenOf>
+__device__ __forceinline__ void plan_body(LenOf len_of, int S, int Hq, int Hkv,
                                           int NHG, int D, int kv_dtype, int NW, char* ws, size_t off_prefix,
                                           size_t off_wplan, size_t off_counters) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -50,7 +45,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   const int chunk = (S + kPlanThreads - 1) / kPlanThreads;
   const int s0 = min(S, tid * chunk), s1 = min(S, s0 + chunk);
   long long local = 0;
-  for (int s = s0; s < s1; ++s) local += ntiles_of(seq_lens[s]);
+  for (int s = s0; s < s1; ++s) local += ntiles_of(len_of(s));
   // block exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5;
   long long incl = local;
@@ -77,7 +72,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   for (int s = s0; s < s1; ++s) {
     prefix[s] = static_cast<int32_t>(run);
     if (in_smem) sp[s] = static_cast<int32_t>(run);
-    run += ntiles_of(seq_lens[s]);
+    run += ntiles_of(len_of(s));
   }
   const long long total_seq_tiles = total_sh;
   if (tid == 0) {
@@ -106,7 +101,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
     }
     wplan[2 * v] = make_int4(static_cast<int>(a), static_cast<int>(b), lo,
                              static_cast<int>(a - static_cast<long long>(P[lo]) * NHG));
-    wplan[2 * v + 1] = make_int4(seq_lens[lo], 0, 0, 0);  // saves the worker a dependent load
+    wplan[2 * v + 1] = make_int4(len_of(lo), 0, 0, 0);  // saves the worker a dependent load
   }
   if (tid == 0) {
     hdr->num_seqs = S;
@@ -126,14 +121,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int kv_dtype, int NW, char* ws,
                                                             size_t off_prefix, size_t off_wplan,
                                                             size_t off_counters) {
-  plan_body(seq_lens, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix, off_wplan, off_counters);
-}
-
-// Two independent plans in one launch, one per CTA.
-__global__ void __launch_bounds__(kPlanThreads) plan2_kernel(const PlanArgs p0, const PlanArgs p1) {
-  const PlanArgs& p = blockIdx.x == 0 ? p0 : p1;
-  plan_body(p.seq_lens, p.S, p.Hq, p.Hkv, p.NHG, p.D, p.kv_dtype, p.NW, p.ws, p.off_prefix, p.off_wplan,
-            p.off_counters);
+  plan_body([seq_lens](int s) { return seq_lens[s]; }, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix,
+            off_wplan, off_counters);
 }
 
 }  // namespace pkv
@@ -166,12 +155,29 @@ EncodeFn encode_fn() {
 }
 }  // namespace
 
-// Pool viewed as 4-D (d, slot, kv head, block), box (inner, rows, 1, 1).
+// Pool viewed as 4-D (d, slot, kv head, block), box (inner, rows, 1, 1); or,
+// for 16-row boxes of swizzled rows longer than one 128-byte part, as 5-D
+// (inner part of d, slot, part, kv head, block) with one box per tile.
 bool make_pool_map(CUtensorMap* m, const void* pool, int dtype, int D, int B, int Hkv, int N,
                    int box_inner, int box_rows, bool swizzle) {
   EncodeFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t es = dtype == PKV_BF16 ? 2 : 4;
+  if (tile_map_5d(D * static_cast<int>(es), box_inner * static_cast<int>(es), box_rows, swizzle)) {
+    // (inner part of d, slot, part of d, kv head, block): one box fetches all
+    // parts of d of a 16-row tile, part-major, as the 4-D map's boxes would
+    const cuuint64_t parts = static_cast<cuuint64_t>(D / box_inner);
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(box_inner), static_cast<cuuint64_t>(B), parts,
+                          static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[4] = {es * Hkv * D, es * box_inner, es * D, es * Hkv * D * B};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows),
+                         static_cast<cuuint32_t>(parts), 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    5, const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+  }
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(B),
                         static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(N)};
   cuuint64_t strides[3] = {es * Hkv * D, es * D, es * Hkv * D * B};
@@ -511,52 +517,121 @@ CascadeLayout cascade_layout(int32_t S, int32_t NG, int32_t T, int32_t Hq, int32
 
 namespace pkv {
 
-// One block per request s: its group g and member index i, its row of the
-// grouped queries, its suffix table and length; the group's first member also
-// writes the group table and length and zeroes the unused member rows.
-__global__ void cascade_gather_kernel(const char* __restrict__ q, const int32_t* __restrict__ tables,
-                                      int32_t max_blocks, const int32_t* __restrict__ seq_lens, int32_t S,
-                                      const int32_t* __restrict__ group_start,
-                                      const int32_t* __restrict__ prefix_blocks, int32_t NG, int32_t T,
-                                      int32_t row_bytes, int32_t B, char* __restrict__ q_grp,
-                                      int32_t* __restrict__ grp_table, int32_t* __restrict__ grp_len,
-                                      int32_t* __restrict__ suf_table, int32_t* __restrict__ suf_len,
-                                      uint32_t* __restrict__ status) {
-  const int s = blockIdx.x;
-  // group of s: the last g with group_start[g] <= s
-  int lo = 0, hi = NG - 1;
+struct PrepArgs {
+  const char* q;
+  const int32_t* tables;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  int32_t S;
+  const int32_t* group_start;
+  const int32_t* prefix_blocks;
+  int32_t NG, T, row_bytes, B;
+  char* q_grp;
+  int32_t* grp_table;
+  int32_t* grp_len;
+  int32_t* suf_table;
+  int32_t* suf_len;
+  uint32_t* status;       // the call's status word (suffix workspace)
+  uint32_t* pre_status;   // the shared-part pass's status word
+  // the two plans
+  int32_t Hq, Hkv, D, kv_dtype;
+  int32_t s_NHG, s_NW;
+  char* s_ws;
+  size_t s_prefix, s_wplan, s_counters;
+  int32_t g_Hq, g_NHG, g_NW;
+  char* g_ws;
+  size_t g_prefix, g_wplan, g_counters;
+};
+
+// The group of request s (the last g with group_start[g] <= s) and how many
+// leading blocks s shares with it: prefix_blocks[g], or 0 when the claim is
+// not valid for s (member index outside the group, group larger than T,
+// block count out of range, or s shorter than the shared part).  The gather
+// and both plans read the claim this one way.
+__device__ __forceinline__ int shared_blocks_of(const PrepArgs& p, int s, int* g_out, int* i_out) {
+  int lo = 0, hi = p.NG - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (group_start[mid] <= s) lo = mid; else hi = mid - 1;
+    if (p.group_start[mid] <= s) lo = mid; else hi = mid - 1;
   }
-  const int g = lo;
-  const int first = group_start[g], size = group_start[g + 1] - first;
+  const int first = p.group_start[lo], size = p.group_start[lo + 1] - first;
   const int i = s - first;
-  const int pb = prefix_blocks[g];
-  const bool bad = i < 0 || i >= size || size > T || pb < 0 || pb > max_blocks ||
-                   seq_lens[s] < pb * B;
-  if (bad) {
-    if (threadIdx.x == 0) record_status(status, kStatusBadTable);
+  const int pb = p.prefix_blocks[lo];
+  const bool bad = i < 0 || i >= size || size > p.T || pb < 0 || pb > p.max_blocks || p.seq_lens[s] < pb * p.B;
+  *g_out = lo;
+  *i_out = i;
+  return bad ? -1 - pb : pb;  // < 0: not valid (the claim, encoded)
+}
+
+// One launch prepares both passes.  Blocks 0 .. S-1 gather request s: its row
+// of the grouped queries and its own-part table (the group's first member
+// also writes the group table and zeroes unused member rows).  Block S plans
+// the own-part pass over the lengths seq_len - shared tokens, block S + 1 the
+// shared-part pass over each group's shared tokens; they compute those
+// lengths from the claims themselves (and store them for the passes), so
+// nothing in this launch waits for another block.
+// Lengths the two plans see (one functor type, so the plan's shared arrays
+// exist once): a request's own tokens (its length minus the shared part), or
+// a group's shared tokens (0 for an empty group).
+struct CascadeLen {
+  const PrepArgs* p;
+  bool group;
+  __device__ int operator()(int x) const {
+    int g, i;
+    if (!group) {
+      const int pb = shared_blocks_of(*p, x, &g, &i);
+      return p->seq_lens[x] - (pb > 0 ? pb : 0) * p->B;
+    }
+    const int first = p->group_start[x];
+    if (p->group_start[x + 1] <= first) return 0;
+    const int pb = shared_blocks_of(*p, first, &g, &i);
+    return (pb > 0 ? pb : 0) * p->B;
   }
-  const int pbs = bad ? 0 : pb;
-  const int mi = (i >= 0 && i < T) ? i : 0;
+};
+
+__global__ void __launch_bounds__(kPlanThreads) cascade_prep_kernel(const PrepArgs p) {
+  const int blk = blockIdx.x;
+  if (blk >= p.S) {
+    const bool group = blk == p.S + 1;
+    const CascadeLen len{&p, group};
+    if (group) {
+      // only the shared-part pass records into its status word, and it runs
+      // after this launch: clear it here
+      if (threadIdx.x == 0) *p.pre_status = 0u;
+      plan_body(len, p.NG, p.g_Hq, p.Hkv, p.g_NHG, p.D, p.kv_dtype, p.g_NW, p.g_ws, p.g_prefix, p.g_wplan,
+                p.g_counters);
+      for (int g = threadIdx.x; g < p.NG; g += blockDim.x) p.grp_len[g] = len(g);
+    } else {
+      plan_body(len, p.S, p.Hq, p.Hkv, p.s_NHG, p.D, p.kv_dtype, p.s_NW, p.s_ws, p.s_prefix, p.s_wplan,
+                p.s_counters);
+      for (int s = threadIdx.x; s < p.S; s += blockDim.x) p.suf_len[s] = len(s);
+    }
+    return;
+  }
+  const int s = blk;
+  int g, i;
+  const int pbc = shared_blocks_of(p, s, &g, &i);
+  if (pbc < 0) {
+    if (threadIdx.x == 0) record_status(p.status, kStatusBadTable);
+  }
+  const int pbs = pbc < 0 ? 0 : pbc;
+  const int first = p.group_start[g], size = p.group_start[g + 1] - first;
+  const int mi = (i >= 0 && i < p.T) ? i : 0;
   // query row: q[s] -> q_grp[g][mi]
-  const uint4* src = reinterpret_cast<const uint4*>(q + size_t(s) * row_bytes);
-  uint4* dst = reinterpret_cast<uint4*>(q_grp + (size_t(g) * T + mi) * row_bytes);
-  for (int u = threadIdx.x; u < row_bytes / 16; u += blockDim.x) dst[u] = src[u];
-  const int32_t* row = tables + size_t(s) * max_blocks;
-  const int32_t* lead = tables + size_t(first) * max_blocks;
-  for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) {
-    suf_table[size_t(s) * max_blocks + j] = j + pbs < max_blocks ? row[j + pbs] : -1;
-    if (j < pbs && row[j] != lead[j]) record_status(status, kStatusBadTable);  // not shared after all
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + size_t(s) * p.row_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(p.q_grp + (size_t(g) * p.T + mi) * p.row_bytes);
+  for (int u = threadIdx.x; u < p.row_bytes / 16; u += blockDim.x) dst[u] = src[u];
+  const int32_t* row = p.tables + size_t(s) * p.max_blocks;
+  const int32_t* lead = p.tables + size_t(first) * p.max_blocks;
+  for (int j = threadIdx.x; j < p.max_blocks; j += blockDim.x) {
+    p.suf_table[size_t(s) * p.max_blocks + j] = j + pbs < p.max_blocks ? row[j + pbs] : -1;
+    if (j < pbs && row[j] != lead[j]) record_status(p.status, kStatusBadTable);  // not shared after all
   }
-  if (threadIdx.x == 0) suf_len[s] = seq_lens[s] - pbs * B;
   if (i == 0) {
-    for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) grp_table[size_t(g) * max_blocks + j] = row[j];
-    if (threadIdx.x == 0) grp_len[g] = pbs * B;
-    for (int m = size; m < T; ++m) {
-      uint4* z = reinterpret_cast<uint4*>(q_grp + (size_t(g) * T + m) * row_bytes);
-      for (int u = threadIdx.x; u < row_bytes / 16; u += blockDim.x) z[u] = make_uint4(0, 0, 0, 0);
+    for (int j = threadIdx.x; j < p.max_blocks; j += blockDim.x) p.grp_table[size_t(g) * p.max_blocks + j] = row[j];
+    for (int m = size; m < p.T; ++m) {
+      uint4* z = reinterpret_cast<uint4*>(p.q_grp + (size_t(g) * p.T + m) * p.row_bytes);
+      for (int u = threadIdx.x; u < p.row_bytes / 16; u += blockDim.x) z[u] = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -567,6 +642,9 @@ __global__ void cascade_combine_kernel(const float* __restrict__ o_p, const floa
                                        const int32_t* __restrict__ group_start, int32_t NG, int32_t T,
                                        int32_t S, int32_t Hq, int32_t D, void* out, int32_t out_dtype,
                                        uint32_t* __restrict__ status, const uint32_t* __restrict__ pre_status) {
+  // launched during the shared-part pass's tail: wait until it (and the
+  // own-part pass before it) completed and their results are visible
+  grid_dependency_wait();
   const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid == 0 && lane == 0 && *pre_status) record_status(status, *pre_status);
@@ -636,29 +714,21 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(workspace);
   const int32_t row_bytes = num_q_heads * head_dim * (kv_dtype == PKV_BF16 ? 2 : 4);
-  // The suffix workspace leads: its status word is the call's own.  The
-  // shared-part pass records faults in its own sub-workspace, whose word the
-  // combine kernel folds into the call's; clear both, so a fault of an earlier
-  // call (or an uninitialised workspace) is never reported again.
+  // The suffix workspace leads: its status word is the call's own; clear it
+  // before anything of this call can record a fault.  The shared-part
+  // pass's word is cleared by the preparation launch (the pass runs after
+  // it); the combine folds it into the call's.
   cudaError_t e = cudaMemsetAsync(w + c.suf_ws, 0, sizeof(uint32_t), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(w + c.pre_ws, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return host::cuda_fail(e);
-  cascade_gather_kernel<<<num_seqs, 128, 0, st>>>(
-      static_cast<const char*>(q), block_tables, max_blocks_per_seq, seq_lens, num_seqs, group_start,
-      prefix_blocks, num_groups, max_group, row_bytes, block_size, w + c.q_grp,
-      reinterpret_cast<int32_t*>(w + c.grp_table), reinterpret_cast<int32_t*>(w + c.grp_len),
-      reinterpret_cast<int32_t*>(w + c.suf_table), reinterpret_cast<int32_t*>(w + c.suf_len),
-      reinterpret_cast<uint32_t*>(w + c.suf_ws));
-  rc = host::check_launch();
-  if (rc != PKV_OK) return rc;
-  // both plans in one launch
-  auto plan_args = [&](const Geometry& g, const int32_t* lens, char* pws) {
-    return PlanArgs{lens, g.S, g.Hq, g.Hkv, g.NHG, g.D, g.dtype, g.NW, pws,
-                    g.lay.prefix, g.lay.wplan, g.lay.counters};
-  };
-  plan2_kernel<<<2, kPlanThreads, 0, st>>>(
-      plan_args(c.gs, reinterpret_cast<const int32_t*>(w + c.suf_len), w + c.suf_ws),
-      plan_args(c.gp, reinterpret_cast<const int32_t*>(w + c.grp_len), w + c.pre_ws));
+  PrepArgs pa{static_cast<const char*>(q), block_tables, max_blocks_per_seq, seq_lens, num_seqs, group_start,
+              prefix_blocks, num_groups, max_group, row_bytes, block_size, w + c.q_grp,
+              reinterpret_cast<int32_t*>(w + c.grp_table), reinterpret_cast<int32_t*>(w + c.grp_len),
+              reinterpret_cast<int32_t*>(w + c.suf_table), reinterpret_cast<int32_t*>(w + c.suf_len),
+              reinterpret_cast<uint32_t*>(w + c.suf_ws), reinterpret_cast<uint32_t*>(w + c.pre_ws),
+              num_q_heads, num_kv_heads, head_dim, kv_dtype,
+              c.gs.NHG, c.gs.NW, w + c.suf_ws, c.gs.lay.prefix, c.gs.lay.wplan, c.gs.lay.counters,
+              c.gp.Hq, c.gp.NHG, c.gp.NW, w + c.pre_ws, c.gp.lay.prefix, c.gp.lay.wplan, c.gp.lay.counters};
+  cascade_prep_kernel<<<num_seqs + 2, kPlanThreads, 0, st>>>(pa);
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
   // own-part pass: each request over its own blocks
@@ -681,11 +751,23 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  cascade_combine_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
-      reinterpret_cast<const float*>(w + c.o_p), reinterpret_cast<const float*>(w + c.lse_p),
-      reinterpret_cast<const float*>(w + c.o_s), reinterpret_cast<const float*>(w + c.lse_s), group_start,
-      num_groups, max_group, num_seqs, num_q_heads, head_dim, out, out_dtype,
-      reinterpret_cast<uint32_t*>(w + c.suf_ws), reinterpret_cast<const uint32_t*>(w + c.pre_ws));
+  // a programmatic dependent launch: its blocks are resident during the
+  // shared-part pass's tail and start as soon as it completes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(threads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, cascade_combine_kernel, reinterpret_cast<const float*>(w + c.o_p),
+                         reinterpret_cast<const float*>(w + c.lse_p), reinterpret_cast<const float*>(w + c.o_s),
+                         reinterpret_cast<const float*>(w + c.lse_s), static_cast<const int32_t*>(group_start),
+                         num_groups, max_group, num_seqs, num_q_heads, head_dim, out, out_dtype,
+                         reinterpret_cast<uint32_t*>(w + c.suf_ws), reinterpret_cast<const uint32_t*>(w + c.pre_ws));
+  if (e != cudaSuccess) return host::cuda_fail(e);
   return host::check_launch();
 }
 

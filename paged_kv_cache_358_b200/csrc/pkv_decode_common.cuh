@@ -112,6 +112,14 @@ PKV_DEVINL void store1(void* out, int out_dtype, size_t off, float v) {
 
 PKV_DEVINL int ntiles_of(int len) { return len > 0 ? (len + kTile - 1) / kTile : 0; }
 
+// Whether the pools are read through a 5-D tensor map whose one box is a
+// whole 16-row tile with every 128-byte part of its rows (swizzled rows of
+// more than one part, block size >= 16); otherwise a 4-D map, one box per
+// part and block.
+__host__ __device__ __forceinline__ bool tile_map_5d(int row_bytes, int part_bytes, int box_rows, bool swizzle) {
+  return swizzle && box_rows == kTile && row_bytes > part_bytes;
+}
+
 // Worker that owns flattened tile t when T tiles are split over NW workers
 // (worker v owns [floor(v T / NW), floor((v+1) T / NW))).
 PKV_DEVINL int owner_of(long long t, long long T, int NW) {

@@ -401,21 +401,31 @@ __global__ void __launch_bounds__(W * 32, CPS)
         if (newpair) load_q(st, s, head);
       }
       const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
-      // A runtime loop over the tile's boxes (one for block sizes >= 16): an
-      // unrolled loop over the four a tile can have put four boxes' worth of
-      // predicated copy instructions and their operand moves into every tile
-      // (about 5 us more per 32 x 4096 layer, measured).
-#pragma unroll 1
-      for (int b = 0; b < nbox; ++b) {
-        const int phys = e[6 + b];
+      if (tile_map_5d(Core::ROWB, Core::kChunkRowBytes, box_rows, Core::kSwizzle)) {
+        // one 5-D box per tile: all 128-byte parts of its 16 rows (two copy
+        // instructions per tile instead of four; 0.5 us less per layer, measured)
+        const int phys = e[6];
         if (phys >= 0) {
+          tma_load_5d(smem_u32(stage + Core::kKOff), &maps.k, 0, slot0, 0, head, phys, bar, pol);
+          tma_load_5d(smem_u32(stage + Core::kVOff), &maps.v, 0, slot0, 0, head, phys, bar, pol);
+        }
+      } else {
+        // A runtime loop over the tile's boxes: an unrolled loop over the
+        // four a tile can have put four boxes' worth of predicated copy
+        // instructions and their operand moves into every tile (about 5 us
+        // more per 32 x 4096 layer, measured).
+#pragma unroll 1
+        for (int b = 0; b < nbox; ++b) {
+          const int phys = e[6 + b];
+          if (phys >= 0) {
 #pragma unroll
-          for (int c = 0; c < Core::kChunks; ++c) {
-            const uint32_t off = c * Core::kChunkBytes + b * box_bytes;
-            tma_load_4d(smem_u32(stage + Core::kKOff + off), &maps.k, c * Core::kBoxInner, slot0, head,
-                        phys, bar, pol);
-            tma_load_4d(smem_u32(stage + Core::kVOff + off), &maps.v, c * Core::kBoxInner, slot0, head,
-                        phys, bar, pol);
+            for (int c = 0; c < Core::kChunks; ++c) {
+              const uint32_t off = c * Core::kChunkBytes + b * box_bytes;
+              tma_load_4d(smem_u32(stage + Core::kKOff + off), &maps.k, c * Core::kBoxInner, slot0, head,
+                          phys, bar, pol);
+              tma_load_4d(smem_u32(stage + Core::kVOff + off), &maps.v, c * Core::kBoxInner, slot0, head,
+                          phys, bar, pol);
+            }
           }
         }
       }

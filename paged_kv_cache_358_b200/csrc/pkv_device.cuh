@@ -119,6 +119,17 @@ PKV_DEVINL void tma_load_4d(uint32_t dst, const void* tmap, int32_t c0, int32_t 
       : "memory");
 }
 
+// 5-D tiled TMA load global -> shared, completing on an mbarrier.
+PKV_DEVINL void tma_load_5d(uint32_t dst, const void* tmap, int32_t c0, int32_t c1, int32_t c2,
+                            int32_t c3, int32_t c4, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar),
+      "l"(policy)
+      : "memory");
+}
+
 // Contiguous bulk copy global -> shared (size and both addresses 16-B aligned).
 PKV_DEVINL void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
