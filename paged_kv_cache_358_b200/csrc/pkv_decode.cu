@@ -548,13 +548,15 @@ struct PrepArgs {
 // not valid for s (member index outside the group, group larger than T,
 // block count out of range, or s shorter than the shared part).  The gather
 // and both plans read the claim this one way.
-__device__ __forceinline__ int shared_blocks_of(const PrepArgs& p, int s, int* g_out, int* i_out) {
+// gs: group_start, or its copy in shared memory.
+__device__ __forceinline__ int shared_blocks_of(const PrepArgs& p, const int32_t* gs, int s, int* g_out,
+                                                int* i_out) {
   int lo = 0, hi = p.NG - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (p.group_start[mid] <= s) lo = mid; else hi = mid - 1;
+    if (gs[mid] <= s) lo = mid; else hi = mid - 1;
   }
-  const int first = p.group_start[lo], size = p.group_start[lo + 1] - first;
+  const int first = gs[lo], size = gs[lo + 1] - first;
   const int i = s - first;
   const int pb = p.prefix_blocks[lo];
   const bool bad = i < 0 || i >= size || size > p.T || pb < 0 || pb > p.max_blocks || p.seq_lens[s] < pb * p.B;
@@ -568,54 +570,68 @@ __device__ __forceinline__ int shared_blocks_of(const PrepArgs& p, int s, int* g
 // also writes the group table and zeroes unused member rows).  Block S plans
 // the own-part pass over the lengths seq_len - shared tokens, block S + 1 the
 // shared-part pass over each group's shared tokens; they compute those
-// lengths from the claims themselves (and store them for the passes), so
-// nothing in this launch waits for another block.
-// Lengths the two plans see (one functor type, so the plan's shared arrays
-// exist once): a request's own tokens (its length minus the shared part), or
-// a group's shared tokens (0 for an empty group).
+// lengths from the claims themselves, store them for the passes and plan
+// from the stored values, so nothing in this launch waits for another block.
+// Every block first copies group_start to shared memory (when it has at most
+// kPrepSmemGroups groups): the group of a request is then a search in shared
+// memory instead of a chain of dependent global loads.
+constexpr int kPrepSmemGroups = 2048;
+
+// Lengths the two plans see: a request's own tokens (its length minus the
+// shared part), or a group's shared tokens (0 for an empty group).
 struct CascadeLen {
   const PrepArgs* p;
+  const int32_t* gs;  // group_start or its shared-memory copy
   bool group;
   __device__ int operator()(int x) const {
     int g, i;
     if (!group) {
-      const int pb = shared_blocks_of(*p, x, &g, &i);
+      const int pb = shared_blocks_of(*p, gs, x, &g, &i);
       return p->seq_lens[x] - (pb > 0 ? pb : 0) * p->B;
     }
-    const int first = p->group_start[x];
-    if (p->group_start[x + 1] <= first) return 0;
-    const int pb = shared_blocks_of(*p, first, &g, &i);
+    const int first = gs[x];
+    if (gs[x + 1] <= first) return 0;
+    const int pb = shared_blocks_of(*p, gs, first, &g, &i);
     return (pb > 0 ? pb : 0) * p->B;
   }
 };
 
 __global__ void __launch_bounds__(kPlanThreads) cascade_prep_kernel(const PrepArgs p) {
+  __shared__ int32_t gs_sh[kPrepSmemGroups + 1];
+  const bool gs_in_smem = p.NG <= kPrepSmemGroups;
+  if (gs_in_smem)
+    for (int g = threadIdx.x; g <= p.NG; g += blockDim.x) gs_sh[g] = p.group_start[g];
+  __syncthreads();
+  const int32_t* gs = gs_in_smem ? gs_sh : p.group_start;
   const int blk = blockIdx.x;
   if (blk >= p.S) {
     const bool group = blk == p.S + 1;
-    const CascadeLen len{&p, group};
+    const CascadeLen len{&p, gs, group};
+    int32_t* lens = group ? p.grp_len : p.suf_len;
+    const int n = group ? p.NG : p.S;
+    // only the shared-part pass records into its status word, and it runs
+    // after this launch: clear it here
+    if (group && threadIdx.x == 0) *p.pre_status = 0u;
+    for (int x = threadIdx.x; x < n; x += blockDim.x) lens[x] = len(x);
+    __syncthreads();  // the plan reads the stored lengths (this block's writes)
+    const auto stored = [lens](int x) { return lens[x]; };
     if (group) {
-      // only the shared-part pass records into its status word, and it runs
-      // after this launch: clear it here
-      if (threadIdx.x == 0) *p.pre_status = 0u;
-      plan_body(len, p.NG, p.g_Hq, p.Hkv, p.g_NHG, p.D, p.kv_dtype, p.g_NW, p.g_ws, p.g_prefix, p.g_wplan,
+      plan_body(stored, p.NG, p.g_Hq, p.Hkv, p.g_NHG, p.D, p.kv_dtype, p.g_NW, p.g_ws, p.g_prefix, p.g_wplan,
                 p.g_counters);
-      for (int g = threadIdx.x; g < p.NG; g += blockDim.x) p.grp_len[g] = len(g);
     } else {
-      plan_body(len, p.S, p.Hq, p.Hkv, p.s_NHG, p.D, p.kv_dtype, p.s_NW, p.s_ws, p.s_prefix, p.s_wplan,
+      plan_body(stored, p.S, p.Hq, p.Hkv, p.s_NHG, p.D, p.kv_dtype, p.s_NW, p.s_ws, p.s_prefix, p.s_wplan,
                 p.s_counters);
-      for (int s = threadIdx.x; s < p.S; s += blockDim.x) p.suf_len[s] = len(s);
     }
     return;
   }
   const int s = blk;
   int g, i;
-  const int pbc = shared_blocks_of(p, s, &g, &i);
+  const int pbc = shared_blocks_of(p, gs, s, &g, &i);
   if (pbc < 0) {
     if (threadIdx.x == 0) record_status(p.status, kStatusBadTable);
   }
   const int pbs = pbc < 0 ? 0 : pbc;
-  const int first = p.group_start[g], size = p.group_start[g + 1] - first;
+  const int first = gs[g], size = gs[g + 1] - first;
   const int mi = (i >= 0 && i < p.T) ? i : 0;
   // query row: q[s] -> q_grp[g][mi]
   const uint4* src = reinterpret_cast<const uint4*>(p.q + size_t(s) * p.row_bytes);
