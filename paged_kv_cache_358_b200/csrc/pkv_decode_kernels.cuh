@@ -124,6 +124,113 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
   }
 }
 
+// ---------------------------------------------------------------------------
+// Merge of the split pairs of a 16-column launch, as a kernel of its own
+// launched right behind the partition kernel (a programmatic dependent
+// launch).  With 16 columns a pair's partial states are 8 KB per piece, and
+// one warp merging ~6 of them needs about nine dependent L2 round trips
+// (about 30,000 cycles, measured), run at the very end of the launch by one
+// CTA per pair while every other SM idles.  Here one warp per (pair, column)
+// merges its column: the pieces' m and l, then one batch of loads of their o
+// slices, all independent, over the whole GPU.  Same rule as merge_pair:
+//   M = max_u m_u,  l = sum_u 2^(m_u - M) l_u,  o = sum_u 2^(m_u - M) o_u / l.
+// ---------------------------------------------------------------------------
+template <int D, int G, bool MULTI>
+__global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, int check_Hq, int check_dtype) {
+  constexpr int PS = part_stride(G, D);
+  constexpr int PER = D / 32;  // output elements per lane
+  constexpr int UB = 8;        // pieces whose o slices are loaded together
+  if (threadIdx.x == 0) grid_launch_dependents();
+  // the partition kernel before this one wrote the partial states
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
+  // a plan for another shape: the partition kernel recorded the mismatch
+  if (__ldcg(&hdr->planned) != 1 || __ldcg(&hdr->num_seqs) != a.num_seqs ||
+      __ldcg(&hdr->num_q_heads) != check_Hq || __ldcg(&hdr->num_kv_heads) != a.num_kv_heads ||
+      __ldcg(&hdr->head_dim) != D || __ldcg(&hdr->kv_dtype) != check_dtype ||
+      __ldcg(&hdr->num_workers) != a.num_workers || __ldcg(&hdr->head_groups) != a.head_groups)
+    return;
+  const long long TT = __ldcg(&hdr->total_tiles);
+  const int NW = a.num_workers, NHG = a.head_groups;
+  if (wid >= static_cast<long long>(a.num_seqs) * NHG * G) return;
+  const long long pp = wid / G;  // pair index s * NHG + hg
+  const int c = static_cast<int>(wid % G);
+  const int s = static_cast<int>(pp / NHG), hg = static_cast<int>(pp % NHG);
+  const int T = MULTI ? a.num_q_tokens : 1;
+  const int Gq = MULTI ? a.num_q_heads / a.num_kv_heads : G;
+  const int ncols = MULTI ? T * Gq : G;
+  if (c >= ncols) return;
+  const int nt = ntiles_of(__ldcg(a.seq_lens + s));
+  if (nt == 0) return;  // zeros, written by the partition kernel
+  const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + a.off_prefix);
+  const long long pstart = static_cast<long long>(__ldcg(prefix + s)) * NHG + static_cast<long long>(hg) * nt;
+  if (pstart + nt > TT) return;  // lengths changed since the plan (recorded by the partition kernel)
+  const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + nt - 1, TT, NW);
+  if (v0 == v1) return;  // the whole pair was in one CTA, which wrote it
+  const float* partials = reinterpret_cast<const float*>(a.ws + a.off_partials);
+  auto slot = [&](int u) { return partials + static_cast<size_t>(u + pp) * PS; };
+  // CTAs without tiles (fewer tiles than workers) hold no state
+  auto valid = [&](int u) { return TT >= NW || range_begin(u, TT, NW) < range_begin(u + 1, TT, NW); };
+  // the pieces' maxima and sums: lane j takes pieces v0 + j, v0 + j + 32, ...
+  float M = -INFINITY;
+  for (int u = v0 + lane; u <= v1; u += 32)
+    if (valid(u)) M = fmaxf(M, __ldcg(slot(u) + G * D + c));
+#pragma unroll
+  for (int msk = 16; msk > 0; msk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, msk));
+  // under the causal mask a column no piece saw a token for keeps M = -inf:
+  // subtract 0 there, so every weight is 0
+  const float Ms = (MULTI && M == -INFINITY) ? 0.f : M;
+  float L = 0.f;
+  for (int u = v0 + lane; u <= v1; u += 32)
+    if (valid(u)) L += exp2f(__ldcg(slot(u) + G * D + c) - Ms) * __ldcg(slot(u) + G * D + G + c);
+#pragma unroll
+  for (int msk = 16; msk > 0; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  for (int u0 = v0; u0 <= v1; u0 += 32) {
+    const int u = u0 + lane;
+    const float w = (u <= v1 && valid(u)) ? exp2f(__ldcg(slot(u) + G * D + c) - Ms) : 0.f;
+    const int nb = v1 - u0 + 1 < 32 ? v1 - u0 + 1 : 32;
+    for (int j0 = 0; j0 < nb; j0 += UB) {
+      // UB loads in flight; pieces past the batch read piece v0 with weight 0
+      float vals[UB][PER];
+#pragma unroll
+      for (int j = 0; j < UB; ++j) {
+        const int uj = j0 + j < nb ? u0 + j0 + j : v0;
+        const float* src = slot(uj) + c * D + lane * PER;
+#pragma unroll
+        for (int i = 0; i < PER; i += 4 <= PER ? 4 : PER) {
+          if constexpr (PER >= 4) {
+            const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
+            vals[j][i] = f.x; vals[j][i + 1] = f.y; vals[j][i + 2] = f.z; vals[j][i + 3] = f.w;
+          } else {
+            const float2 f = __ldcg(reinterpret_cast<const float2*>(src + i));
+            vals[j][i] = f.x; vals[j][i + 1] = f.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < UB; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+        const float ww = j0 + j < nb ? wj : 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] = fmaf(ww, vals[j][i], acc[i]);
+      }
+    }
+  }
+  const OutMap om{(static_cast<size_t>(s) * T * a.num_q_heads + static_cast<size_t>(hg) * Gq) * D,
+                  static_cast<size_t>(a.num_q_heads) * D, Gq, D, ncols};
+  const float inv = MULTI ? (L > 0.f ? 1.f / L : 0.f) : 1.f / L;  // 0: nothing attended
+  if constexpr (MULTI) {
+    if (lane == 0) om.put_lse(a.lse, c, M, L);
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) store1(a.out, a.out_dtype, om.row(c) + lane * PER + i, acc[i] * inv);
+}
+
 // After a bounded wait on tile k expired: stop computing and issue no new
 // copies, but give the copies already issued into the warp's ring (tiles
 // k .. k + depth - 1) a last short wait each before the CTA exits, so none
@@ -483,6 +590,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
     float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
     Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
+    // 16 columns: merge_split_kernel, launched behind this kernel, merges the
+    // pieces (no counting in)
+    if constexpr (G == 16) return;
     // Count this CTA in for (request, KV head).  The pair's counter holds two
     // fields: the low 16 bits count pieces that ended their CTA's range, the
     // high 16 bits the one piece a range can hold before that (the tail of a
@@ -644,14 +754,42 @@ int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_
   return host::check_launch();
 }
 
+// The merge kernel of a 16-column launch, as a programmatic dependent launch
+// behind the partition kernel: one warp per (pair, column).
+template <int D, int G, bool MULTI>
+int launch_merge(const Geometry& geo, const DecodeArgs& args, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(args.num_seqs) * args.head_groups * G;
+  if (warps == 0) return PKV_OK;
+  constexpr int kThreads = 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((warps * 32 + kThreads - 1) / kThreads));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // the plan's head count (padded to the column group for several query tokens)
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, merge_split_kernel<D, G, MULTI>, args, geo.Hq, geo.dtype);
+  if (e != cudaSuccess) return host::cuda_fail(e);
+  return host::check_launch();
+}
+
 template <class Core, int G>
 int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, const void* v,
                 cudaStream_t stream) {
   constexpr int WPS = (Core::ROWB >= 512) ? 4 : 8;
+  constexpr int D = Core::ROWB / Core::ESZ;
   if (geo.HG != 1) return PKV_ERR_INVALID;
-  if (args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads || args.lse != nullptr)
-    return launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream);
-  return launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
+  const bool multi = args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads || args.lse != nullptr;
+  const int rc = multi ? launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream)
+                       : launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
+  if constexpr (G == 16) {
+    if (rc == PKV_OK)
+      return multi ? launch_merge<D, G, true>(geo, args, stream) : launch_merge<D, G, false>(geo, args, stream);
+  }
+  return rc;
 }
 
 // One (storage type, head_dim): dispatch on the group size and the core.
