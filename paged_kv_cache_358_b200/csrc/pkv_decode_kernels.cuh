@@ -145,14 +145,6 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
-  // a plan for another shape: the partition kernel recorded the mismatch
-  if (__ldcg(&hdr->planned) != 1 || __ldcg(&hdr->num_seqs) != a.num_seqs ||
-      __ldcg(&hdr->num_q_heads) != check_Hq || __ldcg(&hdr->num_kv_heads) != a.num_kv_heads ||
-      __ldcg(&hdr->head_dim) != D || __ldcg(&hdr->kv_dtype) != check_dtype ||
-      __ldcg(&hdr->num_workers) != a.num_workers || __ldcg(&hdr->head_groups) != a.head_groups)
-    return;
-  const long long TT = __ldcg(&hdr->total_tiles);
   const int NW = a.num_workers, NHG = a.head_groups;
   if (wid >= static_cast<long long>(a.num_seqs) * NHG * G) return;
   const long long pp = wid / G;  // pair index s * NHG + hg
@@ -162,28 +154,46 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   const int Gq = MULTI ? a.num_q_heads / a.num_kv_heads : G;
   const int ncols = MULTI ? T * Gq : G;
   if (c >= ncols) return;
-  const int nt = ntiles_of(__ldcg(a.seq_lens + s));
-  if (nt == 0) return;  // zeros, written by the partition kernel
+  // one round trip: the plan's header, the request's length and tile offset
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + a.off_prefix);
-  const long long pstart = static_cast<long long>(__ldcg(prefix + s)) * NHG + static_cast<long long>(hg) * nt;
-  if (pstart + nt > TT) return;  // lengths changed since the plan (recorded by the partition kernel)
+  const int planned = __ldcg(&hdr->planned), h_s = __ldcg(&hdr->num_seqs), h_hq = __ldcg(&hdr->num_q_heads);
+  const int h_hkv = __ldcg(&hdr->num_kv_heads), h_d = __ldcg(&hdr->head_dim), h_dt = __ldcg(&hdr->kv_dtype);
+  const int h_nw = __ldcg(&hdr->num_workers), h_nhg = __ldcg(&hdr->head_groups);
+  const long long TT = __ldcg(&hdr->total_tiles);
+  const int len = __ldcg(a.seq_lens + s);
+  const int pre = __ldcg(prefix + s);
+  // a plan for another shape: the partition kernel recorded the mismatch
+  if (planned != 1 || h_s != a.num_seqs || h_hq != check_Hq || h_hkv != a.num_kv_heads || h_d != D ||
+      h_dt != check_dtype || h_nw != NW || h_nhg != NHG)
+    return;
+  const int nt = ntiles_of(len);
+  if (nt == 0) return;  // zeros, written by the partition kernel
+  const long long pstart = static_cast<long long>(pre) * NHG + static_cast<long long>(hg) * nt;
+  if (pstart < 0 || pstart + nt > TT) return;  // lengths changed since the plan (recorded there)
   const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + nt - 1, TT, NW);
   if (v0 == v1) return;  // the whole pair was in one CTA, which wrote it
   const float* partials = reinterpret_cast<const float*>(a.ws + a.off_partials);
   auto slot = [&](int u) { return partials + static_cast<size_t>(u + pp) * PS; };
   // CTAs without tiles (fewer tiles than workers) hold no state
   auto valid = [&](int u) { return TT >= NW || range_begin(u, TT, NW) < range_begin(u + 1, TT, NW); };
-  // the pieces' maxima and sums: lane j takes pieces v0 + j, v0 + j + 32, ...
-  float M = -INFINITY;
-  for (int u = v0 + lane; u <= v1; u += 32)
+  // the pieces' maxima and sums: lane j holds pieces v0 + j, v0 + j + 32, ...
+  // (up to 32 pieces in registers, the common case; more are re-read)
+  float mj = -INFINITY, lj = 0.f;
+  if (v0 + lane <= v1 && valid(v0 + lane)) {
+    mj = __ldcg(slot(v0 + lane) + G * D + c);
+    lj = __ldcg(slot(v0 + lane) + G * D + G + c);
+  }
+  float M = mj;
+  for (int u = v0 + 32 + lane; u <= v1; u += 32)
     if (valid(u)) M = fmaxf(M, __ldcg(slot(u) + G * D + c));
 #pragma unroll
   for (int msk = 16; msk > 0; msk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, msk));
   // under the causal mask a column no piece saw a token for keeps M = -inf:
   // subtract 0 there, so every weight is 0
   const float Ms = (MULTI && M == -INFINITY) ? 0.f : M;
-  float L = 0.f;
-  for (int u = v0 + lane; u <= v1; u += 32)
+  float L = exp2f(mj - Ms) * lj;
+  for (int u = v0 + 32 + lane; u <= v1; u += 32)
     if (valid(u)) L += exp2f(__ldcg(slot(u) + G * D + c) - Ms) * __ldcg(slot(u) + G * D + G + c);
 #pragma unroll
   for (int msk = 16; msk > 0; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
@@ -192,7 +202,8 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   for (int u0 = v0; u0 <= v1; u0 += 32) {
     const int u = u0 + lane;
-    const float w = (u <= v1 && valid(u)) ? exp2f(__ldcg(slot(u) + G * D + c) - Ms) : 0.f;
+    float w = exp2f(mj - Ms);  // 0 for an empty or missing piece (mj = -inf)
+    if (u0 != v0) w = (u <= v1 && valid(u)) ? exp2f(__ldcg(slot(u) + G * D + c) - Ms) : 0.f;
     const int nb = v1 - u0 + 1 < 32 ? v1 - u0 + 1 : 32;
     for (int j0 = 0; j0 < nb; j0 += UB) {
       // UB loads in flight; pieces past the batch read piece v0 with weight 0
