@@ -398,7 +398,8 @@ class DecodeStep:
                 pkv.kv_append(k_new[i], v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
                 self.launches += 1
             if self.shared_prefix:
-                # memset + gather + both plans + two attention passes + combine
+                # preparation (gather + both plans), two attention passes, the
+                # shared pass's merge and the combine: five kernels (and a memset)
                 pkv.paged_decode_attn_shared_prefix(q[i], self.k_pools[i], self.v_pools[i], self.tab_d,
                                                     self.len_d, self.group_start, self.prefix_blocks,
                                                     self.max_group, self.wl.scale, out=out[i],

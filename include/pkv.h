@@ -91,7 +91,10 @@ const char* pkv_last_cuda_error(void);
  * (request, KV head) split across CTAs is finished by the last CTA to reach
  * it, which merges the partial states
  * ([P2] exercise "逻辑顺序没错，为什么 attention 输出还是错？": the states merge,
- * per-block outputs do not).
+ * per-block outputs do not).  With 16 grouped columns (G = 16, or several
+ * query tokens whose columns make 16) the pieces are merged instead by a
+ * second, short launch behind the first: one warp per (request, KV head,
+ * column).
  *
  * Arguments (all device pointers unless stated):
  *   q             [num_seqs][num_q_heads][head_dim], kv_dtype
@@ -245,11 +248,12 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  *                 differ inside the shared part or groups that break the
  *                 rules above (PKV_ERR_BAD_TABLE: the output is then not
  *                 meaningful)
- * Other arguments as pkv_paged_decode_attn.  A 4-byte memset and four
+ * Other arguments as pkv_paged_decode_attn.  A 4-byte memset and five
  * launches: the preparation (gather of the grouped queries and tables, and
  * both plans), the own-part pass, the shared-part pass (the members' queries
  * are the columns of one launch; it starts during the own-part pass's tail),
- * and the combine (started during the shared-part pass's tail). */
+ * the merge of its split pieces (16 columns) and the combine (each started
+ * during the tail of the launch before it). */
 size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_blocks_per_seq);
