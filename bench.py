@@ -73,7 +73,7 @@ def parse():
     p.add_argument("--unfused", action="store_true",
                    help="append with a separate kv_append launch instead of folding it into attention")
     p.add_argument("--pool-copies", type=int, default=None,
-                   help="pool copies the multi_query extra rotates over (fewer: smaller profiling captures)")
+                   help="pool copies the multi_query and prefix_cow extras rotate over (fewer: smaller profiling captures)")
     p.add_argument("--layers", type=int, default=32,
                    help="layers per step (32 for the workload; fewer only for small profiling captures)")
     return p.parse_args()
@@ -633,7 +633,7 @@ def _time_decode(pkv, torch, q, pools, tables, lens, scale, ws, reps):
     return e0.elapsed_time(e1) * 1000 / reps
 
 
-def prefix_cow_measurement(reps: int = 20):
+def prefix_cow_measurement(reps: int = 20, copies: int = 8):
     """Shared prompts: 64 groups x 4 branches fork one 2008-token prompt (full
     blocks shared, the 8-token tail copied on the first append) and append 256
     tokens each; one layer (H_q 16, H_kv 4, d 128, bf16, B 16).  Reports the
@@ -670,7 +670,7 @@ def prefix_cow_measurement(reps: int = 20):
     gen = torch.Generator(device="cuda")
     gen.manual_seed(7)
     pools = [(torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16),
-              torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16)) for _ in range(8)]
+              torch.randn((N, B, Hkv, D), generator=gen, device="cuda", dtype=torch.bfloat16)) for _ in range(copies)]
     q = torch.randn((S, Hq, D), generator=gen, device="cuda", dtype=torch.bfloat16)
     ws = pkv.new_workspace(S, Hq, Hkv, D)
     us = _time_decode(pkv, torch, q, pools, td, ld, wl.scale, ws, reps)
@@ -984,6 +984,8 @@ def main():
     if args.extra is not None:
         if args.extra == "multi_query" and args.pool_copies:
             res = multi_query_measurement(copies=args.pool_copies)
+        elif args.extra == "prefix_cow" and args.pool_copies:
+            res = prefix_cow_measurement(copies=args.pool_copies)
         else:
             res = EXTRAS[args.extra]()
         print(json.dumps({args.extra: res}), flush=True)

@@ -206,11 +206,13 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
     if (u0 != v0) w = (u <= v1 && valid(u)) ? exp2f(__ldcg(slot(u) + G * D + c) - Ms) : 0.f;
     const int nb = v1 - u0 + 1 < 32 ? v1 - u0 + 1 : 32;
     for (int j0 = 0; j0 < nb; j0 += UB) {
-      // UB loads in flight; pieces past the batch read piece v0 with weight 0
+      // UB loads in flight.  Pieces past the batch, and CTAs without tiles
+      // (their slots were never written and may hold any bits, NaN included),
+      // read piece v0 instead, which always holds a state, with weight 0.
       float vals[UB][PER];
 #pragma unroll
       for (int j = 0; j < UB; ++j) {
-        const int uj = j0 + j < nb ? u0 + j0 + j : v0;
+        const int uj = (j0 + j < nb && valid(u0 + j0 + j)) ? u0 + j0 + j : v0;
         const float* src = slot(uj) + c * D + lane * PER;
 #pragma unroll
         for (int i = 0; i < PER; i += 4 <= PER ? 4 : PER) {

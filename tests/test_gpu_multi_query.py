@@ -129,3 +129,40 @@ def test_multi_query_rejects_unsupported_shapes():
                                           2, 32, 8, 128, 16, wl.pool_blocks, wl.scale, pkv.BF16,
                                           out.data_ptr(), pkv.BF16, ws.data_ptr(), ws.numel(), None)
         assert rc == pkv.Status.INVALID
+
+
+@pytest.mark.parametrize("T,Hq,Hkv", [
+    (1, 32, 2),     # single token, 16 grouped heads: the split pieces merged by their own launch
+    (4, 8, 2),      # 4 tokens of 4 heads: 16 columns, causal
+    (1, 8, 2),      # 4 columns: merged by the last CTA to finish a pair
+])
+def test_stale_workspace_bytes_never_reach_the_output(T, Hq, Hkv):
+    """Fewer tiles than CTAs: most CTAs own no tile, so a split pair's pieces
+    sit on CTAs with empty ones between them, whose partial-state slots are
+    never written.  With the workspace filled with 0xFF bytes (NaN as fp32)
+    before the call, the outputs must equal those of a zeroed workspace
+    bit for bit, and the oracle's.  (The first word, the status that faults
+    accumulate in until pkv_decode_status reads it, is read and cleared once
+    after the fill; every other byte stays stale.)"""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    D, B = 128, 16
+    lengths = (37, 91, 128, 201, 511, 0, 1, 17)
+    wl, hb, q = _case(T, Hq, Hkv, D, B, "bf16", lengths, seed=90 + T)
+    db = device_batch(hb)
+    S = len(lengths)
+    n = pkv.lib().pkv_multi_query_workspace_bytes(S, T, Hq, Hkv, D)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = torch.full((int(n),), fill, dtype=torch.uint8, device="cuda")
+        pkv.decode_status(ws)
+        outs.append(pkv.paged_attn_multi_query(torch_from_host(q), db.k_pool, db.v_pool, db.tables, db.seq_lens,
+                                               wl.scale, out_dtype=torch.float32, workspace=ws))
+        assert pkv.decode_status(ws) == pkv.Status.OK
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+    got = as_f64(outs[1])
+    assert np.all(np.isfinite(got))
+    assert np.abs(got - _ref(hb, q)).max() <= TOL_BF16
