@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + nt - 1, TT, NW);
   if (v0 == v1) return;  // the whole pair was in one CTA, which wrote it
   const float* partials = reinterpret_cast<const float*>(a.ws + a.off_partials);
+  // workers are one-warp CTAs (head group 1, which launch_core requires), so
+  // worker u's piece of the pair is slot u + pp
   auto slot = [&](int u) { return partials + static_cast<size_t>(u + pp) * PS; };
   // CTAs without tiles (fewer tiles than workers) hold no state
   auto valid = [&](int u) { return TT >= NW || range_begin(u, TT, NW) < range_begin(u + 1, TT, NW); };
