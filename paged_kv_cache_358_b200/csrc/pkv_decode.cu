@@ -159,13 +159,14 @@ EncodeFn encode_fn() {
 // for 16-row boxes of swizzled rows longer than one 128-byte part, as 5-D
 // (inner part of d, slot, part, kv head, block) with one box per tile.
 bool make_pool_map(CUtensorMap* m, const void* pool, int dtype, int D, int B, int Hkv, int N,
-                   int box_inner, int box_rows, bool swizzle) {
+                   int box_inner, int box_rows, bool swizzle, int block_rows) {
   EncodeFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t es = dtype == PKV_BF16 ? 2 : 4;
-  if (tile_map_5d(D * static_cast<int>(es), box_inner * static_cast<int>(es), box_rows, swizzle)) {
+  if (tile_map_5d(D * static_cast<int>(es), box_inner * static_cast<int>(es), box_rows, swizzle, block_rows)) {
     // (inner part of d, slot, part of d, kv head, block): one box fetches all
-    // parts of d of a 16-row tile, part-major, as the 4-D map's boxes would
+    // parts of d of a 16-row tile, part-major, as the 4-D map's boxes would,
+    // or of one block's box_rows rows
     const cuuint64_t parts = static_cast<cuuint64_t>(D / box_inner);
     cuuint64_t dims[5] = {static_cast<cuuint64_t>(box_inner), static_cast<cuuint64_t>(B), parts,
                           static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(N)};

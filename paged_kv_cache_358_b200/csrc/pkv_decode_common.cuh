@@ -112,12 +112,14 @@ PKV_DEVINL void store1(void* out, int out_dtype, size_t off, float v) {
 
 PKV_DEVINL int ntiles_of(int len) { return len > 0 ? (len + kTile - 1) / kTile : 0; }
 
-// Whether the pools are read through a 5-D tensor map whose one box is a
-// whole 16-row tile with every 128-byte part of its rows (swizzled rows of
-// more than one part, block size >= 16); otherwise a 4-D map, one box per
-// part and block.
-__host__ __device__ __forceinline__ bool tile_map_5d(int row_bytes, int part_bytes, int box_rows, bool swizzle) {
-  return swizzle && box_rows == kTile && row_bytes > part_bytes;
+// Whether the pools are read through a 5-D tensor map whose box holds every
+// 128-byte part of its rows (swizzled rows of more than one part): one box
+// per 16-row tile (block size >= 16), or one per block when the tile core
+// lays a tile out block by block (block_rows: its rows per block box, 4);
+// otherwise a 4-D map, one box per part and block.
+__host__ __device__ __forceinline__ bool tile_map_5d(int row_bytes, int part_bytes, int box_rows, bool swizzle,
+                                                     int block_rows) {
+  return swizzle && row_bytes > part_bytes && (box_rows == kTile || box_rows == block_rows);
 }
 
 // Worker that owns flattened tile t when T tiles are split over NW workers

@@ -54,6 +54,7 @@ struct FmaCore {
   static constexpr int kChunkRowBytes = ROWB;
   static constexpr int kChunkBytes = TILEB;
   static constexpr bool kSwizzle = false;
+  static constexpr int kBlockRows = kTile;  // boxes of up to 16 rows, [row] layout
   static constexpr int kScratchBytes = round_up((kTile * G + G) * 4, 16);
 
   static_assert(U >= 8 && U <= 32, "row must be 128, 256 or 512 bytes");

@@ -523,13 +523,27 @@ __global__ void __launch_bounds__(W * 32, CPS)
         if (newpair) load_q(st, s, head);
       }
       const int slot0 = Bsz >= kTile ? (j * kTile) % Bsz : 0;
-      if (tile_map_5d(Core::ROWB, Core::kChunkRowBytes, box_rows, Core::kSwizzle)) {
-        // one 5-D box per tile: all 128-byte parts of its 16 rows (two copy
-        // instructions per tile instead of four; 0.5 us less per layer, measured)
-        const int phys = e[6];
-        if (phys >= 0) {
-          tma_load_5d(smem_u32(stage + Core::kKOff), &maps.k, 0, slot0, 0, head, phys, bar, pol);
-          tma_load_5d(smem_u32(stage + Core::kVOff), &maps.v, 0, slot0, 0, head, phys, bar, pol);
+      if (tile_map_5d(Core::ROWB, Core::kChunkRowBytes, box_rows, Core::kSwizzle, Core::kBlockRows)) {
+        if (box_rows == kTile) {
+          // one 5-D box per tile: all 128-byte parts of its 16 rows (two copy
+          // instructions per tile instead of four; 0.5 us less per layer, measured)
+          const int phys = e[6];
+          if (phys >= 0) {
+            tma_load_5d(smem_u32(stage + Core::kKOff), &maps.k, 0, slot0, 0, head, phys, bar, pol);
+            tma_load_5d(smem_u32(stage + Core::kVOff), &maps.v, 0, slot0, 0, head, phys, bar, pol);
+          }
+        } else {
+          // one box per block, all parts of its rows, block after block
+          // (the core's [block][part][row] layout; each box 1 KiB-aligned)
+#pragma unroll 1
+          for (int b = 0; b < nbox; ++b) {
+            const int phys = e[6 + b];
+            if (phys >= 0) {
+              const uint32_t off = b * box_rows * Core::ROWB;
+              tma_load_5d(smem_u32(stage + Core::kKOff + off), &maps.k, 0, 0, 0, head, phys, bar, pol);
+              tma_load_5d(smem_u32(stage + Core::kVOff + off), &maps.v, 0, 0, 0, head, phys, bar, pol);
+            }
+          }
         }
       } else {
         // A runtime loop over the tile's boxes: an unrolled loop over the
@@ -724,7 +738,7 @@ struct Geometry {
 extern int g_kernel_choice;  // 0 auto, 1 CUDA-core tiles, 2 tensor-core tiles (bf16)
 
 bool make_pool_map(CUtensorMap* m, const void* pool, int dtype, int D, int B, int Hkv, int N,
-                   int box_inner, int box_rows, bool swizzle);
+                   int box_inner, int box_rows, bool swizzle, int block_rows);
 
 template <class Core, int G, int W, int CPS, bool MULTI>
 int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_pool, const void* v_pool,
@@ -734,10 +748,12 @@ int launch_partition(const Geometry& geo, const DecodeArgs& args, const void* k_
   static_assert(SM::kTotal <= kSmemPerSM, "shared memory budget");
   TmaMaps maps;
   const int box_rows = args.block_size < kTile ? args.block_size : kTile;
+  // a core that lays tiles out block by block reads only boxes of its rows
+  if (Core::kBlockRows != kTile && box_rows != Core::kBlockRows) return PKV_ERR_INVALID;
   if (!make_pool_map(&maps.k, k_pool, geo.dtype, geo.D, args.block_size, geo.Hkv, args.num_blocks,
-                     Core::kBoxInner, box_rows, Core::kSwizzle) ||
+                     Core::kBoxInner, box_rows, Core::kSwizzle, Core::kBlockRows) ||
       !make_pool_map(&maps.v, v_pool, geo.dtype, geo.D, args.block_size, geo.Hkv, args.num_blocks,
-                     Core::kBoxInner, box_rows, Core::kSwizzle)) {
+                     Core::kBoxInner, box_rows, Core::kSwizzle, Core::kBlockRows)) {
     host::set_error("cuTensorMapEncodeTiled failed");
     return PKV_ERR_CUDA;
   }
@@ -814,14 +830,23 @@ int run_decode(const Geometry& geo, const DecodeArgs& args, const void* k, const
   auto per_g = [&](auto gc) -> int {
     constexpr int G = decltype(gc)::value;
     // tensor-core tiles for bf16: up to 8 columns with the tokens in the MMA's
-    // M dimension; 16 columns (head_dim <= 128) with the columns in M
+    // M dimension; 16 columns (head_dim <= 128) with the columns in M.  Block
+    // size 4 (head_dim >= 128): tiles laid out block by block.
     if constexpr (sizeof(T) == 2 && G <= 8) {
       if (args.block_size >= 8 && g_kernel_choice != 1)
         return launch_core<MmaCore<D, G>, G>(geo, args, k, v, stream);
+      if constexpr (D >= 128) {
+        if (args.block_size == 4 && g_kernel_choice != 1)
+          return launch_core<MmaCore<D, G, 4>, G>(geo, args, k, v, stream);
+      }
     }
     if constexpr (sizeof(T) == 2 && G == 16 && D <= 128) {
       if (args.block_size >= 8 && g_kernel_choice != 1)
         return launch_core<MmaCoreM16<D>, G>(geo, args, k, v, stream);
+      if constexpr (D >= 128) {
+        if (args.block_size == 4 && g_kernel_choice != 1)
+          return launch_core<MmaCoreM16<D, 4>, G>(geo, args, k, v, stream);
+      }
     }
     return launch_core<FmaCore<T, D, G>, G>(geo, args, k, v, stream);
   };

@@ -62,7 +62,13 @@ PKV_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int D, int G>
+// SB: rows of one block per TMA box.  kTile (block size >= 16, or 8 through
+// one box per 128-byte part and block): a tile holds each 128-byte part of
+// its 16 rows together, [part][row].  4 (block size 4): one box per block
+// brings all parts of its 4 rows, so a tile is [block][part][row]; each box
+// still starts on a 1 KiB boundary (head_dim >= 128), as the 128-byte
+// swizzle's pattern needs.
+template <int D, int G, int SB = kTile>
 struct MmaCore {
   static constexpr int ESZ = 2;
   static constexpr int ROWB = D * ESZ;
@@ -94,8 +100,19 @@ struct MmaCore {
   };
 
   // Byte offset of (row t, 16-byte unit) inside a swizzled tile.
+  static constexpr int kBlockRows = SB;  // rows per box when a tile spans several blocks
+  static_assert(SB == kTile || (SB == 4 && NCH >= 2), "4-row boxes start on 1 KiB boundaries only with >= 2 parts");
+
   static PKV_DEVINL uint32_t swz(int t, int unit) {
-    return static_cast<uint32_t>((unit >> 3) * CHUNKB + t * 128 + (((unit & 7) ^ (t & 7)) << 4));
+    if constexpr (SB == kTile) {
+      return static_cast<uint32_t>((unit >> 3) * CHUNKB + t * 128 + (((unit & 7) ^ (t & 7)) << 4));
+    } else {
+      // row r of block b, part p: the swizzle pattern follows the row's
+      // position in the 1 KiB-aligned box, p * SB + r
+      const int b = t / SB, r = t % SB, p = unit >> 3;
+      return static_cast<uint32_t>(b * (SB * ROWB) + p * (SB * 128) + r * 128 +
+                                   (((unit & 7) ^ ((p * SB + r) & 7)) << 4));
+    }
   }
 
   // Byte offset of 16-byte unit `unit` of token row t in a K or V tile.
@@ -281,9 +298,10 @@ struct MmaCore {
 // 16 scores sit in the 4 lanes of one quad (2 shuffle levels for its max and
 // sum).  K is read with ldmatrix as the B operand, V with ldmatrix.trans.
 // Same shared-memory stage layout as MmaCore (TMA 128-byte swizzle).
-template <int D>
+template <int D, int SB = kTile>
 struct MmaCoreM16 {
-  using Base = MmaCore<D, 8>;  // tile layout, swizzle and output helpers (independent of G)
+  using Base = MmaCore<D, 8, SB>;  // tile layout, swizzle and output helpers (independent of G)
+  static constexpr int kBlockRows = SB;
   static constexpr int G = 16;
   static constexpr int ESZ = Base::ESZ;
   static constexpr int ROWB = Base::ROWB;
