@@ -282,7 +282,10 @@ int pkv_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size
 
 /* Selects the tile kernel for bf16 storage: 0 = automatic (default),
  * 1 = CUDA-core FMA tiles, 2 = tensor-core (mma.sync bf16) tiles.  fp32
- * storage always uses FMA tiles.  Process-wide; for measurement. */
+ * storage always uses FMA tiles, and so do bf16 pools that the tensor-core
+ * tiles do not cover (block size 4 at head_dim 64; 16 grouped columns at
+ * head_dim 256); 0 and 2 pick the tensor-core tiles everywhere else.
+ * Process-wide; for measurement. */
 int pkv_set_decode_kernel(int32_t which);
 
 /* Launch overlap (default 0 = off).  With 1, pkv_paged_decode_attn_run and
