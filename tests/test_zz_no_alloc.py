@@ -4,7 +4,8 @@ pkv_paged_decode_attn_noalloc exists for callers that cannot allocate device
 memory themselves (a plugin whose host runtime owns every device allocation,
 a serving loop that must never call cudaMalloc).  It keeps its scratch in an
 array built into the library, shared by every call on a device.  This test
-calls it through the C ABI twice in a row, on two different batches, and
+calls it through the C ABI on three different batches in a row (one with 16
+grouped heads per KV head, whose split pieces a second launch merges), and
 checks each result against pkv_paged_decode_attn with a caller workspace and
 against the float64 oracle, so a second call that picked up state left by the
 first would fail.  It also checks that a batch whose stated workspace size is
@@ -37,13 +38,19 @@ def _noalloc(db, wl, out):
     return rc
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def test_noalloc_matches_workspace_entry_point_on_successive_calls():
     import torch
 
     import paged_kv_cache_358_b200 as pkv
 
+    # 16 grouped heads per KV head: the 16-column tiles, whose split pieces
+    # the second launch merges from the same built-in scratch
+    lens16 = tuple(list(W.workload("mixed_512").lengths)[:200])
+    wl16 = W.DecodeWorkload("g16", 1, 32, 2, 128, 16, "bf16", lens16,
+                            pool_blocks=sum(-(-n // 16) for n in lens16) + 8, seed=5)
     cases = [(W.workload("mixed_512", block_size=16), list(W.workload("mixed_512").lengths)[:300], 1e-2),
-             (W.workload("tiny"), None, 1e-5)]
+             (W.workload("tiny"), None, 1e-5),
+             (wl16, None, 1e-2)]
     for wl, lengths, tol in cases:
         hb = host_batch(wl, lengths=lengths)
         db = device_batch(hb)
