@@ -4,7 +4,8 @@ A decode step of several layers, each with its own pools, with the new token's
 append folded in, is run twice from the same state: once with ordinary
 launches and once with pkv_set_launch_overlap(1) for every layer after the
 first (the first follows the plan kernel, whose output it reads).  Outputs and pools must be
-bit-identical, and the outputs must match the float64 oracle.
+bit-identical, and the outputs must match the float64 oracle; with 4 and with
+16 grouped heads per KV head.
 """
 import numpy as np
 import pytest
@@ -28,13 +29,21 @@ def _step(pkv, torch, db, qs, kn, vn, slots, pools, scale, ws, out_dtype, overla
     return outs
 
 
-def test_overlap_is_bit_identical_and_matches_oracle():
+@pytest.mark.parametrize("heads", [None, (32, 2)], ids=["g4", "g16"])
+def test_overlap_is_bit_identical_and_matches_oracle(heads):
+    """g4: the 512-request workload's shapes (H_q 32, H_kv 8).  g16: 16 grouped
+    heads per KV head, where each layer is two launches (the partition kernel
+    and the merge of its split pieces), so a layer's partition kernel starts
+    during the tail of the previous layer's merge launch."""
     import torch
 
     import paged_kv_cache_358_b200 as pkv
 
     wl = W.workload("mixed_512", block_size=16)
     lengths = [int(n) + 1 for n in wl.lengths[:96]]          # history + the new token
+    if heads is not None:
+        wl = W.DecodeWorkload("overlap_g16", 1, heads[0], heads[1], wl.head_dim, 16, "bf16", tuple(lengths),
+                              pool_blocks=sum(-(-n // 16) for n in lengths) + 8, seed=23)
     hb = host_batch(wl, lengths=lengths, seed=21)
     db = device_batch(hb)
     S, Hq, Hkv, D, B = len(lengths), wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
