@@ -53,6 +53,8 @@ def _ref(hb, q):
     (3, 16, 4, 64, 16, "f32"),     # 12 columns padded to 16, fp32 pools
     (16, 8, 8, 128, 4, "f32"),     # 16 tokens, no grouping, 4-token blocks
     (2, 6, 2, 128, 16, "bf16"),    # a group of 3: 6 columns padded to 8
+    (4, 32, 8, 128, 4, "bf16"),    # 16 columns at block size 4: tiles laid out block by block
+    (2, 16, 4, 128, 4, "bf16"),    # 8 columns at block size 4
 ])
 def test_multi_query_all_outputs(kernel, T, Hq, Hkv, D, B, dtype):
     import torch

@@ -82,6 +82,7 @@ def _build(sizes, prompts, appends, Hq, Hkv, D, B, dtype, seed):
     (16, 4, 128, 16, "bf16", (4, 1, 3, 4, 2)),
     (8, 4, 64, 8, "f32", (3, 2, 1, 3)),
     (32, 8, 128, 16, "bf16", (2, 4, 1)),
+    (16, 4, 128, 4, "bf16", (4, 2, 3)),    # block size 4: tensor-core tiles laid out block by block
 ])
 def test_shared_prefix_matches_oracle_and_plain_decode(Hq, Hkv, D, B, dtype, sizes):
     import torch
