@@ -300,7 +300,10 @@ int pkv_set_decode_kernel(int32_t which);
  * pool the call reads: e.g. layers 2..L of one decode step, each reading its
  * own pool, but not the first layer right after pkv_decode_plan.  The calls
  * that plan themselves (pkv_paged_decode_attn, pkv_paged_attn_multi_query,
- * the allocation-free call) never overlap.  Process-wide; read at launch. */
+ * the allocation-free call) ignore this setting: their attention launch
+ * follows their plan launch as a dependent launch that waits for the plan
+ * before reading anything (only its start-up overlaps the plan's).
+ * Process-wide; read at launch. */
 int pkv_set_launch_overlap(int32_t on);
 
 /* ==========================================================================

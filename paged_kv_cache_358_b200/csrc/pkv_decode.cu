@@ -121,6 +121,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int kv_dtype, int NW, char* ws,
                                                             size_t off_prefix, size_t off_wplan,
                                                             size_t off_counters) {
+  // an attention launch after this one may be scheduled now: it waits for
+  // this kernel before reading the plan
+  if (threadIdx.x == 0) grid_launch_dependents();
   plan_body([seq_lens](int s) { return seq_lens[s]; }, S, Hq, Hkv, NHG, D, kv_dtype, NW, ws, off_prefix,
             off_wplan, off_counters);
 }
@@ -324,7 +327,8 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
-             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr) {
+             int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr,
+             bool after_plan = false) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -365,7 +369,10 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   args.num_q_tokens = num_q_tokens;
   args.causal = causal;
   args.lse = lse;
-  geo.overlap = overlap;
+  // after_plan: a programmatic dependent launch right behind the plan kernel
+  // that writes its plan, waiting for it before reading anything
+  geo.overlap = overlap || after_plan;
+  args.wait_first = after_plan ? 1 : 0;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
   args.v_new = new_slots ? v_new : nullptr;
@@ -432,10 +439,11 @@ int pkv_paged_decode_attn(const void* q, const void* k_pool, const void* v_pool,
   if (num_seqs == 0) return PKV_OK;
   rc = do_plan(geo, seq_lens, workspace, static_cast<cudaStream_t>(stream));
   if (rc != PKV_OK) return rc;
-  // the plan kernel just launched writes what the attention reads first: no overlap
+  // the plan kernel just launched writes what the attention reads first: the
+  // attention waits for it at its very top, its launch overlapping the plan's
   return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                   num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
-                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, 1, false);
+                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, 1, false, 1, nullptr, true);
 }
 
 int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* k_pool, const void* v_pool,
@@ -458,7 +466,8 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
   if (rc != PKV_OK) return rc;
   return run_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                   num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, out, out_dtype,
-                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, num_q_tokens);
+                  workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, num_q_tokens, false, 1, nullptr,
+                  true);
 }
 
 }  // extern "C"

@@ -101,6 +101,10 @@ struct DecodeArgs {
   const int64_t* new_slots;
   void* k_pool;
   void* v_pool;
+  // 1: launched as a dependent of the plan kernel that writes this launch's
+  // plan: wait for it before reading anything (the launch's own start-up
+  // then overlaps the plan kernel instead of following it)
+  int32_t wait_first;
 };
 
 PKV_DEVINL void store1(void* out, int out_dtype, size_t off, float v) {

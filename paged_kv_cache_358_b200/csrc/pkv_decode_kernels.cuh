@@ -321,6 +321,10 @@ __global__ void __launch_bounds__(W * 32, CPS)
   int32_t* bt = reinterpret_cast<int32_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SM::kStages + SM::kScratch + SM::kMeta + SM::kBatchB);
 
+  // A launch behind the plan kernel that writes its plan waits for it first,
+  // and only then lets its own dependents be scheduled, so that they too
+  // start after everything the plan kernel wrote is there.
+  if (a.wait_first) grid_dependency_wait();
   // The next kernel of the stream may be scheduled now; it starts on an SM
   // as this launch's CTAs leave it.
   if (threadIdx.x == 0) grid_launch_dependents();
