@@ -398,13 +398,14 @@ class DecodeStep:
                 pkv.kv_append(k_new[i], v_new[i], self.slots, self.k_pools[i], self.v_pools[i])
                 self.launches += 1
             if self.shared_prefix:
-                # preparation (gather + both plans), two attention passes, the
-                # shared pass's merge and the combine: five kernels (and a memset)
+                # preparation (gather + both plans), two attention passes and
+                # the combine (which merges the shared pass's split pieces):
+                # four kernels (and a memset)
                 pkv.paged_decode_attn_shared_prefix(q[i], self.k_pools[i], self.v_pools[i], self.tab_d,
                                                     self.len_d, self.group_start, self.prefix_blocks,
                                                     self.max_group, self.wl.scale, out=out[i],
                                                     workspace=self.wsp)
-                self.launches += 5
+                self.launches += 4
                 continue
             pkv.set_launch_overlap(self.overlap and i > 0 and self.fused)
             if self.fused:

@@ -248,12 +248,13 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  *                 differ inside the shared part or groups that break the
  *                 rules above (PKV_ERR_BAD_TABLE: the output is then not
  *                 meaningful)
- * Other arguments as pkv_paged_decode_attn.  A 4-byte memset and five
+ * Other arguments as pkv_paged_decode_attn.  A 4-byte memset and four
  * launches: the preparation (gather of the grouped queries and tables, and
  * both plans), the own-part pass, the shared-part pass (the members' queries
- * are the columns of one launch; it starts during the own-part pass's tail),
- * the merge of its split pieces (16 columns) and the combine (each started
- * during the tail of the launch before it). */
+ * are the columns of one launch; it starts during the own-part pass's tail)
+ * and the combine (started during the shared-part pass's tail), which also
+ * merges the shared-part pass's split pieces when that pass has 16 columns
+ * per KV head. */
 size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_blocks_per_seq);

@@ -328,7 +328,7 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
              int32_t kv_dtype, void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
              pkv_stream_t stream, const void* k_new, const void* v_new, const int64_t* new_slots,
              int32_t num_q_tokens = 1, bool overlap = false, int32_t causal = 1, float* lse = nullptr,
-             bool after_plan = false) {
+             bool after_plan = false, bool merge_by_caller = false, DecodeArgs* args_out = nullptr) {
   // T query tokens per request run as more grouped heads over the same KV
   // heads: the columns of a KV head are (query token, grouped head), padded
   // to a power of two.
@@ -373,12 +373,14 @@ int run_impl(const void* q, const void* k_pool, const void* v_pool, const int32_
   // that writes its plan, waiting for it before reading anything
   geo.overlap = overlap || after_plan;
   args.wait_first = after_plan ? 1 : 0;
+  args.merge_by_caller = merge_by_caller ? 1 : 0;
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   args.k_new = new_slots ? k_new : nullptr;
   args.v_new = new_slots ? v_new : nullptr;
   args.new_slots = new_slots;
   args.k_pool = const_cast<void*>(k_pool);
   args.v_pool = const_cast<void*>(v_pool);
+  if (args_out) *args_out = args;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (kv_dtype == PKV_BF16) {
     switch (head_dim) {
@@ -662,12 +664,33 @@ __global__ void __launch_bounds__(kPlanThreads) cascade_prep_kernel(const PrepAr
   }
 }
 
+// A lane's PER consecutive floats of a row (16-byte loads where they fit).
+template <int PER>
+__device__ __forceinline__ void load_row_slice(const float* __restrict__ src, float (&v)[PER]) {
+#pragma unroll
+  for (int i = 0; i < PER; i += (PER >= 4 ? 4 : 2)) {
+    if constexpr (PER >= 4) {
+      const float4 f = *reinterpret_cast<const float4*>(src + i);
+      v[i] = f.x; v[i + 1] = f.y; v[i + 2] = f.z; v[i + 3] = f.w;
+    } else {
+      const float2 f = *reinterpret_cast<const float2*>(src + i);
+      v[i] = f.x; v[i + 1] = f.y;
+    }
+  }
+}
+
 // One warp per (request, query head): combine the two partial results.
-__global__ void cascade_combine_kernel(const float* __restrict__ o_p, const float* __restrict__ lse_p,
+// With 16 columns in the shared-part pass (merge_here), the pieces of its
+// split pairs are merged here, column by column (merge_column), instead of by
+// a launch of their own; its whole pairs were written to o_p / lse_p.
+template <int D>
+__global__ void cascade_combine_kernel(const DecodeArgs sp, int sp_check_hq, int sp_check_dtype, int merge_here,
+                                       const float* __restrict__ o_p, const float* __restrict__ lse_p,
                                        const float* __restrict__ o_s, const float* __restrict__ lse_s,
                                        const int32_t* __restrict__ group_start, int32_t NG, int32_t T,
-                                       int32_t S, int32_t Hq, int32_t D, void* out, int32_t out_dtype,
+                                       int32_t S, int32_t Hq, int32_t Hkv, void* out, int32_t out_dtype,
                                        uint32_t* __restrict__ status, const uint32_t* __restrict__ pre_status) {
+  constexpr int PER = D / 32;  // output elements per lane
   // launched during the shared-part pass's tail: wait until it (and the
   // own-part pass before it) completed and their results are visible
   grid_dependency_wait();
@@ -685,7 +708,26 @@ __global__ void cascade_combine_kernel(const float* __restrict__ o_p, const floa
   i = i < 0 ? 0 : (i >= T ? T - 1 : i);
   const size_t pr = (static_cast<size_t>(lo) * T + i) * Hq + h;  // prefix row
   const size_t sr = static_cast<size_t>(s) * Hq + h;              // suffix row
-  const float lp = lse_p[pr], ls = lse_s[sr];
+  float op[PER], lp = -INFINITY;
+  bool merged = false;
+  if (merge_here) {
+    const int Gq = Hq / Hkv;
+    float M, L, acc[PER];
+    if (merge_column<D, 16, true>(sp, sp_check_hq, sp_check_dtype, lo, h / Gq, i * Gq + h % Gq, lane, M, L, acc)) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) op[e] = acc[e] * inv;
+      lp = L > 0.f ? M + __log2f(L) : -INFINITY;
+      merged = true;
+    }
+  }
+  if (!merged) {
+    lp = lse_p[pr];
+    load_row_slice<PER>(o_p + pr * D + lane * PER, op);
+  }
+  const float ls = lse_s[sr];
+  float os[PER];
+  load_row_slice<PER>(o_s + sr * D + lane * PER, os);
   const float M = fmaxf(lp, ls);
   float wp = 0.f, wsf = 0.f;
   if (M != -INFINITY) {
@@ -694,9 +736,10 @@ __global__ void cascade_combine_kernel(const float* __restrict__ o_p, const floa
   }
   const float den = wp + wsf;
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int d = lane; d < D; d += 32) {
-    const float v = (wp * o_p[pr * D + d] + wsf * o_s[sr * D + d]) * inv;
-    store1(out, out_dtype, sr * D + d, v);
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const float v = (wp * op[e] + wsf * os[e]) * inv;
+    store1(out, out_dtype, sr * D + lane * PER + e, v);
   }
 }
 
@@ -763,6 +806,7 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                 block_size, num_blocks, scale, kv_dtype, w + c.o_s, PKV_F32, w + c.suf_ws, c.gs.lay.total,
                 stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
   if (rc != PKV_OK) return rc;
+  DecodeArgs sp{};  // the shared-part pass's launch arguments, for the combine's merge
   // shared-part pass: groups x members, every member sees the whole shared
   // part.  It may start during the own-part pass's tail (launch overlap):
   // what it reads first -- its plan, the group tables and lengths, the pools
@@ -772,7 +816,7 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                 max_blocks_per_seq, reinterpret_cast<const int32_t*>(w + c.grp_len), num_groups, num_q_heads,
                 num_kv_heads, head_dim, block_size, num_blocks, scale, kv_dtype, w + c.o_p, PKV_F32,
                 w + c.pre_ws, c.gp.lay.total, stream, nullptr, nullptr, nullptr, max_group, true, 0,
-                reinterpret_cast<float*>(w + c.lse_p));
+                reinterpret_cast<float*>(w + c.lse_p), false, /*merge_by_caller=*/true, &sp);
   if (rc != PKV_OK) return rc;
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
   const int threads = 256;
@@ -788,11 +832,22 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, cascade_combine_kernel, reinterpret_cast<const float*>(w + c.o_p),
-                         reinterpret_cast<const float*>(w + c.lse_p), reinterpret_cast<const float*>(w + c.o_s),
-                         reinterpret_cast<const float*>(w + c.lse_s), static_cast<const int32_t*>(group_start),
-                         num_groups, max_group, num_seqs, num_q_heads, head_dim, out, out_dtype,
-                         reinterpret_cast<uint32_t*>(w + c.suf_ws), reinterpret_cast<const uint32_t*>(w + c.pre_ws));
+  // 16 columns in the shared-part pass: its split pairs are merged here
+  const int merge_here = c.gp.G == 16 ? 1 : 0;
+  auto combine = [&](auto kern) {
+    return cudaLaunchKernelEx(&cfg, kern, sp, c.gp.Hq, kv_dtype, merge_here,
+                              reinterpret_cast<const float*>(w + c.o_p), reinterpret_cast<const float*>(w + c.lse_p),
+                              reinterpret_cast<const float*>(w + c.o_s), reinterpret_cast<const float*>(w + c.lse_s),
+                              static_cast<const int32_t*>(group_start), num_groups, max_group, num_seqs,
+                              num_q_heads, num_kv_heads, out, out_dtype, reinterpret_cast<uint32_t*>(w + c.suf_ws),
+                              reinterpret_cast<const uint32_t*>(w + c.pre_ws));
+  };
+  switch (head_dim) {
+    case 64: e = combine(cascade_combine_kernel<64>); break;
+    case 128: e = combine(cascade_combine_kernel<128>); break;
+    case 256: e = combine(cascade_combine_kernel<256>); break;
+    default: return PKV_ERR_INVALID;
+  }
   if (e != cudaSuccess) return host::cuda_fail(e);
   return host::check_launch();
 }

@@ -124,36 +124,21 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
   }
 }
 
-// ---------------------------------------------------------------------------
-// Merge of the split pairs of a 16-column launch, as a kernel of its own
-// launched right behind the partition kernel (a programmatic dependent
-// launch).  With 16 columns a pair's partial states are 8 KB per piece, and
-// one warp merging ~6 of them needs about nine dependent L2 round trips
-// (about 30,000 cycles, measured), run at the very end of the launch by one
-// CTA per pair while every other SM idles.  Here one warp per (pair, column)
-// merges its column: the pieces' m and l, then one batch of loads of their o
-// slices, all independent, over the whole GPU.  Same rule as merge_pair:
-//   M = max_u m_u,  l = sum_u 2^(m_u - M) l_u,  o = sum_u 2^(m_u - M) o_u / l.
-// ---------------------------------------------------------------------------
+// Merge of column c of (request s, KV head `head`) from the pieces of its
+// split pair, as the partition kernel left them in the workspace `a.ws`.
+// Returns false when there is nothing to merge here (the pair was not split,
+// the request is empty, or the plan is for another shape -- which the
+// partition kernel recorded); otherwise M (the max, log2 domain), L (the sum)
+// and the lane's D/32 output elements, not yet divided by L.
 template <int D, int G, bool MULTI>
-__global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, int check_Hq, int check_dtype) {
+__device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, int check_dtype, int s, int head,
+                                             int c, int lane, float& M, float& L, float (&acc)[D / 32]) {
   constexpr int PS = part_stride(G, D);
   constexpr int PER = D / 32;  // output elements per lane
   constexpr int UB = 8;        // pieces whose o slices are loaded together
-  if (threadIdx.x == 0) grid_launch_dependents();
-  // the partition kernel before this one wrote the partial states
-  grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int NW = a.num_workers, NHG = a.head_groups;
-  if (wid >= static_cast<long long>(a.num_seqs) * NHG * G) return;
-  const long long pp = wid / G;  // pair index s * NHG + hg
-  const int c = static_cast<int>(wid % G);
-  const int s = static_cast<int>(pp / NHG), hg = static_cast<int>(pp % NHG);
-  const int T = MULTI ? a.num_q_tokens : 1;
-  const int Gq = MULTI ? a.num_q_heads / a.num_kv_heads : G;
-  const int ncols = MULTI ? T * Gq : G;
-  if (c >= ncols) return;
+  const int hg = head;  // one-warp workers: the head group is the KV head
+  const long long pp = static_cast<long long>(s) * NHG + hg;  // pair index s * NHG + hg
   // one round trip: the plan's header, the request's length and tile offset
   const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + a.off_prefix);
@@ -166,13 +151,13 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   // a plan for another shape: the partition kernel recorded the mismatch
   if (planned != 1 || h_s != a.num_seqs || h_hq != check_Hq || h_hkv != a.num_kv_heads || h_d != D ||
       h_dt != check_dtype || h_nw != NW || h_nhg != NHG)
-    return;
+    return false;
   const int nt = ntiles_of(len);
-  if (nt == 0) return;  // zeros, written by the partition kernel
+  if (nt == 0) return false;  // zeros, written by the partition kernel
   const long long pstart = static_cast<long long>(pre) * NHG + static_cast<long long>(hg) * nt;
-  if (pstart < 0 || pstart + nt > TT) return;  // lengths changed since the plan (recorded there)
+  if (pstart < 0 || pstart + nt > TT) return false;  // lengths changed since the plan (recorded there)
   const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + nt - 1, TT, NW);
-  if (v0 == v1) return;  // the whole pair was in one CTA, which wrote it
+  if (v0 == v1) return false;  // the whole pair was in one CTA, which wrote it
   const float* partials = reinterpret_cast<const float*>(a.ws + a.off_partials);
   // workers are one-warp CTAs (head group 1, which launch_core requires), so
   // worker u's piece of the pair is slot u + pp
@@ -186,7 +171,7 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
     mj = __ldcg(slot(v0 + lane) + G * D + c);
     lj = __ldcg(slot(v0 + lane) + G * D + G + c);
   }
-  float M = mj;
+  M = mj;
   for (int u = v0 + 32 + lane; u <= v1; u += 32)
     if (valid(u)) M = fmaxf(M, __ldcg(slot(u) + G * D + c));
 #pragma unroll
@@ -194,12 +179,11 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
   // under the causal mask a column no piece saw a token for keeps M = -inf:
   // subtract 0 there, so every weight is 0
   const float Ms = (MULTI && M == -INFINITY) ? 0.f : M;
-  float L = exp2f(mj - Ms) * lj;
+  L = exp2f(mj - Ms) * lj;
   for (int u = v0 + 32 + lane; u <= v1; u += 32)
     if (valid(u)) L += exp2f(__ldcg(slot(u) + G * D + c) - Ms) * __ldcg(slot(u) + G * D + G + c);
 #pragma unroll
   for (int msk = 16; msk > 0; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
-  float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   for (int u0 = v0; u0 <= v1; u0 += 32) {
@@ -236,6 +220,40 @@ __global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, in
       }
     }
   }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Merge of the split pairs of a 16-column launch, as a kernel of its own
+// launched right behind the partition kernel (a programmatic dependent
+// launch).  With 16 columns a pair's partial states are 8 KB per piece, and
+// one warp merging ~6 of them needs about nine dependent L2 round trips
+// (about 30,000 cycles, measured), run at the very end of the launch by one
+// CTA per pair while every other SM idles.  Here one warp per (pair, column)
+// merges its column (merge_column): the pieces' m and l, then one batch of
+// loads of their o slices, all independent, over the whole GPU.  Same rule as
+// merge_pair:
+//   M = max_u m_u,  l = sum_u 2^(m_u - M) l_u,  o = sum_u 2^(m_u - M) o_u / l.
+// ---------------------------------------------------------------------------
+template <int D, int G, bool MULTI>
+__global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, int check_Hq, int check_dtype) {
+  constexpr int PER = D / 32;
+  if (threadIdx.x == 0) grid_launch_dependents();
+  // the partition kernel before this one wrote the partial states
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int NHG = a.head_groups;
+  if (wid >= static_cast<long long>(a.num_seqs) * NHG * G) return;
+  const long long pp = wid / G;  // pair index s * NHG + hg
+  const int c = static_cast<int>(wid % G);
+  const int s = static_cast<int>(pp / NHG), hg = static_cast<int>(pp % NHG);
+  const int T = MULTI ? a.num_q_tokens : 1;
+  const int Gq = MULTI ? a.num_q_heads / a.num_kv_heads : G;
+  const int ncols = MULTI ? T * Gq : G;
+  if (c >= ncols) return;
+  float M, L, acc[PER];
+  if (!merge_column<D, G, MULTI>(a, check_Hq, check_dtype, s, hg, c, lane, M, L, acc)) return;
   const OutMap om{(static_cast<size_t>(s) * T * a.num_q_heads + static_cast<size_t>(hg) * Gq) * D,
                   static_cast<size_t>(a.num_q_heads) * D, Gq, D, ncols};
   const float inv = MULTI ? (L > 0.f ? 1.f / L : 0.f) : 1.f / L;  // 0: nothing attended
@@ -821,7 +839,7 @@ int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, cons
   const int rc = multi ? launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream)
                        : launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
   if constexpr (G == 16) {
-    if (rc == PKV_OK)
+    if (rc == PKV_OK && !args.merge_by_caller)
       return multi ? launch_merge<D, G, true>(geo, args, stream) : launch_merge<D, G, false>(geo, args, stream);
   }
   return rc;
