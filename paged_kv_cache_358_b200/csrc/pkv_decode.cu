@@ -609,6 +609,9 @@ struct CascadeLen {
 };
 
 __global__ void __launch_bounds__(kPlanThreads) cascade_prep_kernel(const PrepArgs p) {
+  // The own-part pass behind this launch may be scheduled now: its CTAs
+  // become resident while this launch runs and wait for it at their top.
+  if (threadIdx.x == 0) grid_launch_dependents();
   __shared__ int32_t gs_sh[kPrepSmemGroups + 1];
   const bool gs_in_smem = p.NG <= kPrepSmemGroups;
   if (gs_in_smem)
@@ -681,53 +684,79 @@ __device__ __forceinline__ void load_row_slice(const float* __restrict__ src, fl
 
 // One warp per (request, query head): combine the two partial results.
 // With 16 columns in the shared-part pass (merge_here), the pieces of its
-// split pairs are merged here, column by column (merge_column), instead of by
-// a launch of their own; its whole pairs were written to o_p / lse_p.
+// split pairs are merged here, column by column (merge_span, merge_pieces),
+// instead of by a launch of their own; its whole pairs were written to
+// o_p / lse_p.  Before waiting for the shared-part pass a warp finds its
+// group and its pair's span (caller input and plan, written before that pass
+// began); after it, one round trip loads the own part, the pieces' m and l
+// and their o slices together.
+// 128 threads and at most 72 registers (D <= 128): 28 warps per SM, so one
+// warp per (request, query head) of a 256 x 16 batch is resident at once
+// (with 96 registers the last third waited for a second wave, ~7 us).
+constexpr int kCombineThreads = 128;
+constexpr int kCombineSmemGroups = 4096;  // group_start kept in shared memory below this many groups
 template <int D>
-__global__ void cascade_combine_kernel(const DecodeArgs sp, int sp_check_hq, int sp_check_dtype, int merge_here,
-                                       const float* __restrict__ o_p, const float* __restrict__ lse_p,
-                                       const float* __restrict__ o_s, const float* __restrict__ lse_s,
-                                       const int32_t* __restrict__ group_start, int32_t NG, int32_t T,
-                                       int32_t S, int32_t Hq, int32_t Hkv, void* out, int32_t out_dtype,
-                                       uint32_t* __restrict__ status, const uint32_t* __restrict__ pre_status) {
+__global__ void __launch_bounds__(kCombineThreads, D <= 128 ? 7 : 4)
+    cascade_combine_kernel(const DecodeArgs sp, int sp_check_hq, int sp_check_dtype, int merge_here,
+                           const float* __restrict__ o_p, const float* __restrict__ lse_p,
+                           const float* __restrict__ o_s, const float* __restrict__ lse_s,
+                           const int32_t* __restrict__ group_start, int32_t NG, int32_t T, int32_t S,
+                           int32_t Hq, int32_t Hkv, void* out, int32_t out_dtype, uint32_t* __restrict__ status,
+                           const uint32_t* __restrict__ pre_status) {
   constexpr int PER = D / 32;  // output elements per lane
-  // launched during the shared-part pass's tail: wait until it (and the
-  // own-part pass before it) completed and their results are visible
-  grid_dependency_wait();
+  // group_start is the caller's, and no launch of this call writes it: the
+  // CTAs copy it to shared memory and find each warp's group while the
+  // shared-part pass still runs (they are resident during its tail), instead
+  // of a chain of dependent global loads after it.
+  extern __shared__ int32_t gs_sh[];
+  const bool gs_in_smem = NG < kCombineSmemGroups;
+  if (gs_in_smem)
+    for (int g = threadIdx.x; g <= NG; g += blockDim.x) gs_sh[g] = group_start[g];
+  __syncthreads();
+  const int32_t* gs = gs_in_smem ? gs_sh : group_start;
   const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid == 0 && lane == 0 && *pre_status) record_status(status, *pre_status);
-  if (wid >= static_cast<long long>(S) * Hq) return;
-  const int s = static_cast<int>(wid / Hq), h = static_cast<int>(wid % Hq);
-  int lo = 0, hi = NG - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (group_start[mid] <= s) lo = mid; else hi = mid - 1;
+  const bool active = wid < static_cast<long long>(S) * Hq;
+  int s = 0, h = 0, lo = 0, i = 0;
+  MergeSpan span;
+  bool split = false;
+  if (active) {
+    s = static_cast<int>(wid / Hq);
+    h = static_cast<int>(wid % Hq);
+    int hi = NG - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gs[mid] <= s) lo = mid; else hi = mid - 1;
+    }
+    i = s - gs[lo];
+    i = i < 0 ? 0 : (i >= T ? T - 1 : i);
+    // the shared-part pass's plan was written by the preparation launch
+    if (merge_here) split = merge_span(sp, sp_check_hq, sp_check_dtype, D, lo, h / (Hq / Hkv), span);
   }
-  int i = s - group_start[lo];
-  i = i < 0 ? 0 : (i >= T ? T - 1 : i);
+  // wait until the shared-part pass (and the own-part pass before it)
+  // completed and their results are visible
+  grid_dependency_wait();
+  if (wid == 0 && lane == 0 && *pre_status) record_status(status, *pre_status);
+  if (!active) return;
   const size_t pr = (static_cast<size_t>(lo) * T + i) * Hq + h;  // prefix row
   const size_t sr = static_cast<size_t>(s) * Hq + h;              // suffix row
-  float op[PER], lp = -INFINITY;
-  bool merged = false;
-  if (merge_here) {
-    const int Gq = Hq / Hkv;
-    float M, L, acc[PER];
-    if (merge_column<D, 16, true>(sp, sp_check_hq, sp_check_dtype, lo, h / Gq, i * Gq + h % Gq, lane, M, L, acc)) {
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) op[e] = acc[e] * inv;
-      lp = L > 0.f ? M + __log2f(L) : -INFINITY;
-      merged = true;
-    }
-  }
-  if (!merged) {
-    lp = lse_p[pr];
-    load_row_slice<PER>(o_p + pr * D + lane * PER, op);
-  }
+  // the own part's loads are in flight with the shared part's
   const float ls = lse_s[sr];
   float os[PER];
   load_row_slice<PER>(o_s + sr * D + lane * PER, os);
+  float op[PER], lp;
+  if (split) {
+    const int Gq = Hq / Hkv;
+    float M, L, acc[PER];
+    merge_pieces<D, 16, true>(sp, span, i * Gq + h % Gq, lane, M, L, acc);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) op[e] = acc[e] * inv;
+    lp = L > 0.f ? M + __log2f(L) : -INFINITY;
+  } else {
+    lp = lse_p[pr];
+    load_row_slice<PER>(o_p + pr * D + lane * PER, op);
+  }
   const float M = fmaxf(lp, ls);
   float wp = 0.f, wsf = 0.f;
   if (M != -INFINITY) {
@@ -800,11 +829,13 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   cascade_prep_kernel<<<num_seqs + 2, kPlanThreads, 0, st>>>(pa);
   rc = host::check_launch();
   if (rc != PKV_OK) return rc;
-  // own-part pass: each request over its own blocks
+  // own-part pass: each request over its own blocks; a dependent launch whose
+  // CTAs become resident during the preparation and wait for it at their top
   rc = run_impl(q, k_pool, v_pool, reinterpret_cast<const int32_t*>(w + c.suf_table), max_blocks_per_seq,
                 reinterpret_cast<const int32_t*>(w + c.suf_len), num_seqs, num_q_heads, num_kv_heads, head_dim,
                 block_size, num_blocks, scale, kv_dtype, w + c.o_s, PKV_F32, w + c.suf_ws, c.gs.lay.total,
-                stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s));
+                stream, nullptr, nullptr, nullptr, 1, false, 1, reinterpret_cast<float*>(w + c.lse_s),
+                /*after_plan=*/true);
   if (rc != PKV_OK) return rc;
   DecodeArgs sp{};  // the shared-part pass's launch arguments, for the combine's merge
   // shared-part pass: groups x members, every member sees the whole shared
@@ -819,13 +850,14 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                 reinterpret_cast<float*>(w + c.lse_p), false, /*merge_by_caller=*/true, &sp);
   if (rc != PKV_OK) return rc;
   const long long warps = static_cast<long long>(num_seqs) * num_q_heads;
-  const int threads = 256;
+  const int threads = kCombineThreads;
   const long long blocks = (warps * 32 + threads - 1) / threads;
   // a programmatic dependent launch: its blocks are resident during the
   // shared-part pass's tail and start as soon as it completes
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks));
   cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = num_groups < kCombineSmemGroups ? (num_groups + 1) * sizeof(int32_t) : 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

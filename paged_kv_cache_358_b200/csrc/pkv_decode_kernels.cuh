@@ -124,21 +124,21 @@ __device__ __noinline__ void merge_pair(const float* partials, long long pp, int
   }
 }
 
-// Merge of column c of (request s, KV head `head`) from the pieces of its
-// split pair, as the partition kernel left them in the workspace `a.ws`.
-// Returns false when there is nothing to merge here (the pair was not split,
-// the request is empty, or the plan is for another shape -- which the
-// partition kernel recorded); otherwise M (the max, log2 domain), L (the sum)
-// and the lane's D/32 output elements, not yet divided by L.
-template <int D, int G, bool MULTI>
-__device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, int check_dtype, int s, int head,
-                                             int c, int lane, float& M, float& L, float (&acc)[D / 32]) {
-  constexpr int PS = part_stride(G, D);
-  constexpr int PER = D / 32;  // output elements per lane
-  constexpr int UB = 8;        // pieces whose o slices are loaded together
+// Which workers hold the pieces of the split pair (request s, KV head `head`),
+// from the plan alone (its header, the request's length and tile offset):
+// nothing the partition kernel writes, so a merge may find its span before it
+// waits for that kernel.  Returns false when there is nothing to merge (the
+// pair was not split, the request is empty, or the plan is for another shape
+// -- which the partition kernel recorded).
+struct MergeSpan {
+  long long pp;  // pair index s * NHG + head
+  long long TT;  // tiles of the launch
+  int v0, v1;    // first and last worker holding a piece
+  int NW;
+};
+__device__ __forceinline__ bool merge_span(const DecodeArgs& a, int check_Hq, int check_dtype, int D, int s,
+                                           int head, MergeSpan& m) {
   const int NW = a.num_workers, NHG = a.head_groups;
-  const int hg = head;  // one-warp workers: the head group is the KV head
-  const long long pp = static_cast<long long>(s) * NHG + hg;  // pair index s * NHG + hg
   // one round trip: the plan's header, the request's length and tile offset
   const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + a.off_prefix);
@@ -148,22 +148,62 @@ __device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, 
   const long long TT = __ldcg(&hdr->total_tiles);
   const int len = __ldcg(a.seq_lens + s);
   const int pre = __ldcg(prefix + s);
-  // a plan for another shape: the partition kernel recorded the mismatch
   if (planned != 1 || h_s != a.num_seqs || h_hq != check_Hq || h_hkv != a.num_kv_heads || h_d != D ||
       h_dt != check_dtype || h_nw != NW || h_nhg != NHG)
     return false;
   const int nt = ntiles_of(len);
   if (nt == 0) return false;  // zeros, written by the partition kernel
-  const long long pstart = static_cast<long long>(pre) * NHG + static_cast<long long>(hg) * nt;
+  // one-warp workers: the head group is the KV head
+  const long long pstart = static_cast<long long>(pre) * NHG + static_cast<long long>(head) * nt;
   if (pstart < 0 || pstart + nt > TT) return false;  // lengths changed since the plan (recorded there)
-  const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + nt - 1, TT, NW);
-  if (v0 == v1) return false;  // the whole pair was in one CTA, which wrote it
+  m.v0 = owner_of(pstart, TT, NW);
+  m.v1 = owner_of(pstart + nt - 1, TT, NW);
+  if (m.v0 == m.v1) return false;  // the whole pair was in one CTA, which wrote it
+  m.pp = static_cast<long long>(s) * NHG + head;
+  m.TT = TT;
+  m.NW = NW;
+  return true;
+}
+
+// Merge of column c of a split pair from its pieces, as the partition kernel
+// left them in the workspace `a.ws` (call after waiting for that kernel): M
+// (the max, log2 domain), L (the sum) and the lane's D/32 output elements,
+// not yet divided by L.  One round trip loads every piece's m and l and the o
+// slices of the first UB pieces together (the o loads need no weight); more
+// than UB pieces take one more round trip per UB.
+template <int D, int G, bool MULTI>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs& a, const MergeSpan& m, int c, int lane, float& M,
+                                             float& L, float (&acc)[D / 32]) {
+  constexpr int PS = part_stride(G, D);
+  constexpr int PER = D / 32;  // output elements per lane
+  constexpr int UB = 8;        // pieces whose o slices are loaded together
+  const int v0 = m.v0, v1 = m.v1;
   const float* partials = reinterpret_cast<const float*>(a.ws + a.off_partials);
   // workers are one-warp CTAs (head group 1, which launch_core requires), so
   // worker u's piece of the pair is slot u + pp
-  auto slot = [&](int u) { return partials + static_cast<size_t>(u + pp) * PS; };
+  auto slot = [&](int u) { return partials + static_cast<size_t>(u + m.pp) * PS; };
   // CTAs without tiles (fewer tiles than workers) hold no state
-  auto valid = [&](int u) { return TT >= NW || range_begin(u, TT, NW) < range_begin(u + 1, TT, NW); };
+  auto valid = [&](int u) { return m.TT >= m.NW || range_begin(u, m.TT, m.NW) < range_begin(u + 1, m.TT, m.NW); };
+  // UB o slices in flight.  Pieces past the batch, and CTAs without tiles
+  // (their slots were never written and may hold any bits, NaN included),
+  // read piece v0 instead, which always holds a state, with weight 0.
+  auto load_batch = [&](float (&vals)[UB][PER], int first, int nb) {
+#pragma unroll
+    for (int j = 0; j < UB; ++j) {
+      const int uj = (j < nb && valid(first + j)) ? first + j : v0;
+      const float* src = slot(uj) + c * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; i += 4 <= PER ? 4 : PER) {
+        if constexpr (PER >= 4) {
+          const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
+          vals[j][i] = f.x; vals[j][i + 1] = f.y; vals[j][i + 2] = f.z; vals[j][i + 3] = f.w;
+        } else {
+          const float2 f = __ldcg(reinterpret_cast<const float2*>(src + i));
+          vals[j][i] = f.x; vals[j][i + 1] = f.y;
+        }
+      }
+    }
+  };
   // the pieces' maxima and sums: lane j holds pieces v0 + j, v0 + j + 32, ...
   // (up to 32 pieces in registers, the common case; more are re-read)
   float mj = -INFINITY, lj = 0.f;
@@ -171,6 +211,9 @@ __device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, 
     mj = __ldcg(slot(v0 + lane) + G * D + c);
     lj = __ldcg(slot(v0 + lane) + G * D + G + c);
   }
+  const int nb0 = v1 - v0 + 1 < UB ? v1 - v0 + 1 : UB;
+  float vals[UB][PER];
+  load_batch(vals, v0, nb0);
   M = mj;
   for (int u = v0 + 32 + lane; u <= v1; u += 32)
     if (valid(u)) M = fmaxf(M, __ldcg(slot(u) + G * D + c));
@@ -184,43 +227,30 @@ __device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, 
     if (valid(u)) L += exp2f(__ldcg(slot(u) + G * D + c) - Ms) * __ldcg(slot(u) + G * D + G + c);
 #pragma unroll
   for (int msk = 16; msk > 0; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
+  const float w0 = exp2f(mj - Ms);  // 0 for an empty or missing piece (mj = -inf)
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  auto accumulate = [&](const float (&vals)[UB][PER], float w, int j0, int nb) {
+#pragma unroll
+    for (int j = 0; j < UB; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+      const float ww = j0 + j < nb ? wj : 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(ww, vals[j][i], acc[i]);
+    }
+  };
+  accumulate(vals, w0, 0, nb0);
+  // pieces past the first batch (more than UB of them: rare)
   for (int u0 = v0; u0 <= v1; u0 += 32) {
     const int u = u0 + lane;
-    float w = exp2f(mj - Ms);  // 0 for an empty or missing piece (mj = -inf)
+    float w = w0;
     if (u0 != v0) w = (u <= v1 && valid(u)) ? exp2f(__ldcg(slot(u) + G * D + c) - Ms) : 0.f;
     const int nb = v1 - u0 + 1 < 32 ? v1 - u0 + 1 : 32;
-    for (int j0 = 0; j0 < nb; j0 += UB) {
-      // UB loads in flight.  Pieces past the batch, and CTAs without tiles
-      // (their slots were never written and may hold any bits, NaN included),
-      // read piece v0 instead, which always holds a state, with weight 0.
-      float vals[UB][PER];
-#pragma unroll
-      for (int j = 0; j < UB; ++j) {
-        const int uj = (j0 + j < nb && valid(u0 + j0 + j)) ? u0 + j0 + j : v0;
-        const float* src = slot(uj) + c * D + lane * PER;
-#pragma unroll
-        for (int i = 0; i < PER; i += 4 <= PER ? 4 : PER) {
-          if constexpr (PER >= 4) {
-            const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
-            vals[j][i] = f.x; vals[j][i + 1] = f.y; vals[j][i + 2] = f.z; vals[j][i + 3] = f.w;
-          } else {
-            const float2 f = __ldcg(reinterpret_cast<const float2*>(src + i));
-            vals[j][i] = f.x; vals[j][i + 1] = f.y;
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < UB; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
-        const float ww = j0 + j < nb ? wj : 0.f;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) acc[i] = fmaf(ww, vals[j][i], acc[i]);
-      }
+    for (int j0 = (u0 == v0 ? UB : 0); j0 < nb; j0 += UB) {
+      load_batch(vals, u0 + j0, nb - j0);
+      accumulate(vals, w, j0, nb);
     }
   }
-  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -230,30 +260,40 @@ __device__ __forceinline__ bool merge_column(const DecodeArgs& a, int check_Hq, 
 // one warp merging ~6 of them needs about nine dependent L2 round trips
 // (about 30,000 cycles, measured), run at the very end of the launch by one
 // CTA per pair while every other SM idles.  Here one warp per (pair, column)
-// merges its column (merge_column): the pieces' m and l, then one batch of
-// loads of their o slices, all independent, over the whole GPU.  Same rule as
+// merges its column over the whole GPU: its pair's span from the plan before
+// waiting for the partition kernel (merge_span), then one round trip for the
+// pieces' m and l and o slices together (merge_pieces).  Same rule as
 // merge_pair:
 //   M = max_u m_u,  l = sum_u 2^(m_u - M) l_u,  o = sum_u 2^(m_u - M) o_u / l.
 // ---------------------------------------------------------------------------
+// 128 threads and at most 72 registers (D <= 128): 28 warps per SM, so the
+// 4096 (pair, column) warps of 32 requests x 8 KV heads x 16 columns are all
+// resident at once instead of in two waves.
+constexpr int kMergeThreads = 128;
 template <int D, int G, bool MULTI>
-__global__ void __launch_bounds__(256) merge_split_kernel(const DecodeArgs a, int check_Hq, int check_dtype) {
+__global__ void __launch_bounds__(kMergeThreads, D <= 128 ? 7 : 4)
+    merge_split_kernel(const DecodeArgs a, int check_Hq, int check_dtype) {
   constexpr int PER = D / 32;
   if (threadIdx.x == 0) grid_launch_dependents();
-  // the partition kernel before this one wrote the partial states
-  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int NHG = a.head_groups;
-  if (wid >= static_cast<long long>(a.num_seqs) * NHG * G) return;
   const long long pp = wid / G;  // pair index s * NHG + hg
   const int c = static_cast<int>(wid % G);
   const int s = static_cast<int>(pp / NHG), hg = static_cast<int>(pp % NHG);
   const int T = MULTI ? a.num_q_tokens : 1;
   const int Gq = MULTI ? a.num_q_heads / a.num_kv_heads : G;
   const int ncols = MULTI ? T * Gq : G;
-  if (c >= ncols) return;
+  // the pair's span from the plan, which the plan kernel wrote before the
+  // partition kernel began, while that kernel still runs
+  MergeSpan span;
+  const bool split = wid < static_cast<long long>(a.num_seqs) * NHG * G && c < ncols &&
+                     merge_span(a, check_Hq, check_dtype, D, s, hg, span);
+  // the partition kernel before this one wrote the partial states
+  grid_dependency_wait();
+  if (!split) return;
   float M, L, acc[PER];
-  if (!merge_column<D, G, MULTI>(a, check_Hq, check_dtype, s, hg, c, lane, M, L, acc)) return;
+  merge_pieces<D, G, MULTI>(a, span, c, lane, M, L, acc);
   const OutMap om{(static_cast<size_t>(s) * T * a.num_q_heads + static_cast<size_t>(hg) * Gq) * D,
                   static_cast<size_t>(a.num_q_heads) * D, Gq, D, ncols};
   const float inv = MULTI ? (L > 0.f ? 1.f / L : 0.f) : 1.f / L;  // 0: nothing attended
@@ -641,8 +681,8 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
     float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
     Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
-    // 16 columns: merge_split_kernel, launched behind this kernel, merges the
-    // pieces (no counting in)
+    // 16 columns: a later launch merges the pieces (merge_split_kernel right
+    // behind this kernel, or the shared-prefix call's combine), no counting in
     if constexpr (G == 16) return;
     // Count this CTA in for (request, KV head).  The pair's counter holds two
     // fields: the low 16 bits count pieces that ended their CTA's range, the
@@ -813,10 +853,9 @@ template <int D, int G, bool MULTI>
 int launch_merge(const Geometry& geo, const DecodeArgs& args, cudaStream_t stream) {
   const long long warps = static_cast<long long>(args.num_seqs) * args.head_groups * G;
   if (warps == 0) return PKV_OK;
-  constexpr int kThreads = 256;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((warps * 32 + kThreads - 1) / kThreads));
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3(static_cast<unsigned>((warps * 32 + kMergeThreads - 1) / kMergeThreads));
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

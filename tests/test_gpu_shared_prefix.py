@@ -169,3 +169,36 @@ def test_shared_prefix_rejects_unsupported_groups():
                                                16, 1, 0.1, pkv.BF16, z.data_ptr(), pkv.BF16, z.data_ptr(), 1 << 20,
                                                None)
     assert rc == pkv.Status.INVALID                                              # more groups than requests
+
+
+@pytest.mark.parametrize("fill", [0xFF, 0x7F])
+def test_shared_prefix_16_columns_with_stale_workspace(fill):
+    """16 columns per KV head (4 members x 4 grouped heads): the combine merges
+    the shared-part pass's split pieces itself.  Workspace bytes left by
+    anything else (NaN or huge values) must not reach an output: CTAs without
+    tiles never write their slots, and the merge must not read them.  With 44
+    shared tiles over all workers, most workers own none and every split pair
+    spans many of them."""
+    import torch
+
+    import paged_kv_cache_358_b200 as pkv
+
+    Hq, Hkv, D, B = 16, 4, 128, 16
+    sizes, prompts = (4, 3, 4), (150, 40, 0)
+    S = sum(sizes)
+    appends = [(5 * s) % 17 + 1 for s in range(S)]
+    kp, vp, tables, lens, hk, hv, q, gs = _build(sizes, prompts, appends, Hq, Hkv, D, B, "bf16", seed=11)
+    pb = np.array([p // B for p in prompts], np.int32)
+    ws = pkv.shared_prefix_workspace(S, len(sizes), 4, Hq, Hkv, D, tables.shape[1])
+    scale = 1.0 / np.sqrt(D)
+    ws.fill_(fill)
+    for _ in range(2):   # the second call sees what the first left behind
+        out = pkv.paged_decode_attn_shared_prefix(torch_from_host(q), kp, vp, torch.from_numpy(tables).cuda(),
+                                                  torch.from_numpy(lens).cuda(), torch.from_numpy(gs).cuda(),
+                                                  torch.from_numpy(pb).cuda(), 4, scale,
+                                                  out_dtype=torch.float32, workspace=ws)
+        assert pkv.decode_status(ws) == pkv.Status.OK
+        got = as_f64(out)
+        assert np.all(np.isfinite(got))
+        for s in range(S):
+            assert np.max(np.abs(got[s] - oatt.dense_decode(q[s], hk[s], hv[s], scale))) <= 1e-2, f"request {s}"
