@@ -700,9 +700,6 @@ __global__ void __launch_bounds__(W * 32, CPS)
       if (lane == 0) red_release_gpu_add(reinterpret_cast<unsigned*>(&counters[ctr]), 1u << 16);
       return;
     }
-    int prev = 0;
-    if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[ctr], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
     const int v0 = owner_of(pstart, TT, NW), v1 = owner_of(pstart + pnt - 1, TT, NW);
     int expected = v1 - v0 + 1;  // with TT >= NW every CTA owns at least one tile
     if (TT < NW) {
@@ -712,7 +709,17 @@ __global__ void __launch_bounds__(W * 32, CPS)
     // the pair's last piece is flushed mid-range when its CTA's range goes on
     // past the pair's end
     const int expected_mid = (v1 != v0 && range_begin(v1 + 1, TT, NW) > pstart + pnt) ? 1 : 0;
-    if ((prev & 0xffff) == expected - expected_mid - 1) {
+    // The only piece flushed at a range end (the pair's other piece is the
+    // mid-range one, the common case for short pairs) merges whenever the
+    // mid-range piece counts in, so it counts nothing in itself: no atomic,
+    // and no wait for its own partial writes, which only this warp reads.
+    const bool sole = expected - expected_mid == 1;
+    int prev = 0;
+    if (!sole) {
+      if (lane == 0) prev = atomic_add_acq_rel_gpu(&counters[ctr], 1);
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+    }
+    if (sole || (prev & 0xffff) == expected - expected_mid - 1) {
       if ((prev >> 16) < expected_mid) {
         // bounded wait for the mid-range piece (its CTA is running or about
         // to: it needs nothing from this one)
