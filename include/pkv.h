@@ -250,7 +250,8 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  *                 meaningful)
  * Other arguments as pkv_paged_decode_attn.  A 4-byte memset and four
  * launches: the preparation (gather of the grouped queries and tables, and
- * both plans), the own-part pass, the shared-part pass (the members' queries
+ * both plans), the own-part pass (scheduled during the preparation, waiting
+ * for it at its start), the shared-part pass (the members' queries
  * are the columns of one launch; it starts during the own-part pass's tail)
  * and the combine (started during the shared-part pass's tail), which also
  * merges the shared-part pass's split pieces when that pass has 16 columns
