@@ -92,7 +92,9 @@ const char* pkv_last_cuda_error(void);
  * it, which merges the partial states
  * ([P2] exercise "逻辑顺序没错，为什么 attention 输出还是错？": the states merge,
  * per-block outputs do not).  With 16 grouped columns (G = 16, or several
- * query tokens whose columns make 16) the pieces are merged instead by a
+ * query tokens whose columns make 16), and with 8 in a launch that is not
+ * plain single-token decode (several query tokens, query heads padded to the
+ * column group, or a log-sum-exp output), the pieces are merged instead by a
  * second, short launch behind the first: one warp per (request, KV head,
  * column).
  *
@@ -254,8 +256,10 @@ int pkv_paged_attn_multi_query(const void* q, int32_t num_q_tokens, const void* 
  * for it at its start), the shared-part pass (the members' queries
  * are the columns of one launch; it starts during the own-part pass's tail)
  * and the combine (started during the shared-part pass's tail), which also
- * merges the shared-part pass's split pieces when that pass has 16 columns
- * per KV head. */
+ * merges the shared-part pass's split pieces when that pass has 8 or 16
+ * columns per KV head.  With 8 grouped query heads per KV head the own-part
+ * pass (which writes a log-sum-exp) is followed by its merge launch: five
+ * launches. */
 size_t pkv_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_groups, int32_t max_group,
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_blocks_per_seq);

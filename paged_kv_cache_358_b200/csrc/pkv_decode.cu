@@ -683,8 +683,8 @@ __device__ __forceinline__ void load_row_slice(const float* __restrict__ src, fl
 }
 
 // One warp per (request, query head): combine the two partial results.
-// With 16 columns in the shared-part pass (merge_here), the pieces of its
-// split pairs are merged here, column by column (merge_span, merge_pieces),
+// With 8 or 16 columns (GM) in the shared-part pass (merge_here), the pieces
+// of its split pairs are merged here, column by column (merge_span, merge_pieces),
 // instead of by a launch of their own; its whole pairs were written to
 // o_p / lse_p.  Before waiting for the shared-part pass a warp finds its
 // group and its pair's span (caller input and plan, written before that pass
@@ -695,7 +695,7 @@ __device__ __forceinline__ void load_row_slice(const float* __restrict__ src, fl
 // (with 96 registers the last third waited for a second wave, ~7 us).
 constexpr int kCombineThreads = 128;
 constexpr int kCombineSmemGroups = 4096;  // group_start kept in shared memory below this many groups
-template <int D>
+template <int D, int GM>
 __global__ void __launch_bounds__(kCombineThreads, D <= 128 ? 7 : 4)
     cascade_combine_kernel(const DecodeArgs sp, int sp_check_hq, int sp_check_dtype, int merge_here,
                            const float* __restrict__ o_p, const float* __restrict__ lse_p,
@@ -748,7 +748,7 @@ __global__ void __launch_bounds__(kCombineThreads, D <= 128 ? 7 : 4)
   if (split) {
     const int Gq = Hq / Hkv;
     float M, L, acc[PER];
-    merge_pieces<D, 16, true>(sp, span, i * Gq + h % Gq, lane, M, L, acc);
+    merge_pieces<D, GM, true>(sp, span, i * Gq + h % Gq, lane, M, L, acc);
     const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) op[e] = acc[e] * inv;
@@ -864,8 +864,10 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // 16 columns in the shared-part pass: its split pairs are merged here
-  const int merge_here = c.gp.G == 16 ? 1 : 0;
+  // 8 or 16 columns in the shared-part pass (a general launch: it writes a
+  // log-sum-exp): its split pairs are merged here
+  const int merge_here = (c.gp.G == 16 || c.gp.G == 8) ? 1 : 0;
+  const bool gm8 = c.gp.G == 8;
   auto combine = [&](auto kern) {
     return cudaLaunchKernelEx(&cfg, kern, sp, c.gp.Hq, kv_dtype, merge_here,
                               reinterpret_cast<const float*>(w + c.o_p), reinterpret_cast<const float*>(w + c.lse_p),
@@ -875,9 +877,9 @@ int pkv_paged_decode_attn_shared_prefix(const void* q, const void* k_pool, const
                               reinterpret_cast<const uint32_t*>(w + c.pre_ws));
   };
   switch (head_dim) {
-    case 64: e = combine(cascade_combine_kernel<64>); break;
-    case 128: e = combine(cascade_combine_kernel<128>); break;
-    case 256: e = combine(cascade_combine_kernel<256>); break;
+    case 64: e = gm8 ? combine(cascade_combine_kernel<64, 8>) : combine(cascade_combine_kernel<64, 16>); break;
+    case 128: e = gm8 ? combine(cascade_combine_kernel<128, 8>) : combine(cascade_combine_kernel<128, 16>); break;
+    case 256: e = gm8 ? combine(cascade_combine_kernel<256, 8>) : combine(cascade_combine_kernel<256, 16>); break;
     default: return PKV_ERR_INVALID;
   }
   if (e != cudaSuccess) return host::cuda_fail(e);

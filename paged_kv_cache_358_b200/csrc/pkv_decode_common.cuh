@@ -105,8 +105,9 @@ struct DecodeArgs {
   // plan: wait for it before reading anything (the launch's own start-up
   // then overlaps the plan kernel instead of following it)
   int32_t wait_first;
-  // 1: the caller merges the split pieces of a 16-column launch itself (no
-  // merge launch behind the partition kernel)
+  // 1: the caller merges the split pieces of a launch whose pairs a later
+  // launch merges (merged_by_later_launch) itself: no merge launch behind
+  // the partition kernel
   int32_t merge_by_caller;
 };
 

@@ -304,6 +304,16 @@ __global__ void __launch_bounds__(kMergeThreads, D <= 128 ? 7 : 4)
   for (int i = 0; i < PER; ++i) store1(a.out, a.out_dtype, om.row(c) + lane * PER + i, acc[i] * inv);
 }
 
+// Whether a later launch merges a partition launch's split pairs (instead of
+// the last worker of each pair, at the launch's tail): with 16 columns, and
+// with 8 in the general instantiation (several query tokens, padded columns or
+// a log-sum-exp output).  Single-token 8-column decode keeps the in-kernel
+// merge, which measured faster for it.
+template <int G, bool MULTI>
+constexpr bool merged_by_later_launch() {
+  return G == 16 || (G == 8 && MULTI);
+}
+
 // After a bounded wait on tile k expired: stop computing and issue no new
 // copies, but give the copies already issued into the warp's ring (tiles
 // k .. k + depth - 1) a last short wait each before the CTA exits, so none
@@ -681,9 +691,9 @@ __global__ void __launch_bounds__(W * 32, CPS)
     const long long pp = static_cast<long long>(ps) * NHG + phg;  // pair index
     float* part = partials + (static_cast<size_t>(v + pp) * W + warp) * PS;
     Core::finish(state, false, a.out, a.out_dtype, om, part, lane);
-    // 16 columns: a later launch merges the pieces (merge_split_kernel right
-    // behind this kernel, or the shared-prefix call's combine), no counting in
-    if constexpr (G == 16) return;
+    // a later launch merges the pieces (merge_split_kernel right behind this
+    // kernel, or the shared-prefix call's combine), no counting in
+    if constexpr (merged_by_later_launch<G, MULTI>()) return;
     // Count this CTA in for (request, KV head).  The pair's counter holds two
     // fields: the low 16 bits count pieces that ended their CTA's range, the
     // high 16 bits the one piece a range can hold before that (the tail of a
@@ -884,9 +894,11 @@ int launch_core(const Geometry& geo, const DecodeArgs& args, const void* k, cons
   const bool multi = args.num_q_tokens > 1 || args.num_q_heads != G * args.num_kv_heads || args.lse != nullptr;
   const int rc = multi ? launch_partition<Core, G, 1, WPS, true>(geo, args, k, v, stream)
                        : launch_partition<Core, G, 1, WPS, false>(geo, args, k, v, stream);
+  if (rc != PKV_OK || args.merge_by_caller) return rc;
   if constexpr (G == 16) {
-    if (rc == PKV_OK && !args.merge_by_caller)
-      return multi ? launch_merge<D, G, true>(geo, args, stream) : launch_merge<D, G, false>(geo, args, stream);
+    return multi ? launch_merge<D, G, true>(geo, args, stream) : launch_merge<D, G, false>(geo, args, stream);
+  } else if constexpr (G == 8) {
+    if (multi) return launch_merge<D, G, true>(geo, args, stream);  // merged_by_later_launch<8, true>
   }
   return rc;
 }
