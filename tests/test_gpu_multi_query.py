@@ -136,6 +136,8 @@ def test_multi_query_rejects_unsupported_shapes():
 @pytest.mark.parametrize("T,Hq,Hkv", [
     (1, 32, 2),     # single token, 16 grouped heads: the split pieces merged by their own launch
     (4, 8, 2),      # 4 tokens of 4 heads: 16 columns, causal
+    (2, 8, 2),      # 2 tokens of 4 heads: 8 columns, causal, also merged by their own launch
+    (1, 12, 2),     # 6 heads padded to 8 columns: merged by their own launch
     (1, 8, 2),      # 4 columns: merged by the last CTA to finish a pair
 ])
 def test_stale_workspace_bytes_never_reach_the_output(T, Hq, Hkv):
